@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Benchmark of one Wave Forcing layer-round on B200 through libwf.
+
+A step is one pass of the whole hot path over one layer of one wavefront
+round: wf_publish_kv (3D rotary + paged scatter of every live slot),
+wf_round_attention (M_WF-masked attention of every live slot, with the
+readiness check) and wf_advance_round (page recycling + table rewrite). The
+pool is first driven through pipeline fill so every timed step is a steady
+round. Inputs live in HBM before timing starts; the working set (pool, q, k,
+v, q_rot, out) is larger than the 126 MB L2, so no flush is needed between
+steps.
+
+value = unmasked attention FLOPs of the timed steps / device time of those
+steps (TFLOP/s), summed over ranks (each rank runs an independent replica).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "WF round attention TFLOP/s (unmasked)"
+UNIT = "TFLOP/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="wan13b_bf16")
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- utils
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def source_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def read_traffic(kernel_file):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary, or None
+    when the kernel source has changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(os.path.basename(kernel_file))
+    if not e or e.get("source_sha") != source_sha(kernel_file):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.remove(self.path)
+        if not rows:
+            return None
+        mhz = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(mhz) if mhz else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def unmasked_flops(layout, cfg):
+    """4 * C * (keys visible to the slot) * d * heads summed over live slots:
+    QK^T and PV multiply-adds over unmasked (query, key) pairs only."""
+    total = 0
+    for idx, (kind, chunk, slot, tag, pages) in enumerate(layout):
+        if slot is None:
+            continue
+        total += 4 * cfg.chunk_tokens * (idx + 1) * cfg.chunk_tokens * cfg.head_dim * cfg.num_heads
+    return total
+
+
+def publish_bytes(layout, cfg):
+    """Algorithmic HBM bytes of one publish: read q, k, v and write q_rot, K, V
+    pages (rows of live slots; the zeroed page tail counted as written)."""
+    live = sum(1 for r in layout if r[2] is not None)
+    elt = 2 if cfg.dtype == "bf16" else 4
+    row = cfg.num_heads * cfg.head_dim * elt
+    tail = cfg.pages_per_chunk * cfg.page_tokens - cfg.chunk_tokens
+    return live * (6 * cfg.chunk_tokens * row + 2 * tail * row)
+
+
+# ------------------------------------------------------------------------- our arm
+
+def run_ours(args, ws, rank, local):
+    import torch
+    import wf_inputs
+    from chunk_causal_wavefront_b200 import KVPool, make_config
+
+    cfg = wf_inputs.CONFIGS[args.config]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    steady = cfg.steady_round()
+    total_rounds = steady + args.warmup + args.steps + (0 if args.no_e2e else args.e2e_steps + 2) + 4
+    npages = (cfg.num_stages + 1 + cfg.anchor_chunks + cfg.history_chunks) * cfg.pages_per_chunk
+    pool = KVPool(make_config(num_stages=cfg.num_stages, chunk_tokens=cfg.chunk_tokens,
+                              num_heads=cfg.num_heads, head_dim=cfg.head_dim,
+                              anchor_chunks=cfg.anchor_chunks, history_chunks=cfg.history_chunks,
+                              page_tokens=cfg.page_tokens, num_layers=1, dtype=cfg.dtype,
+                              rope=cfg.rope, frames_per_chunk=cfg.frames_per_chunk,
+                              grid_h=cfg.grid_h, grid_w=cfg.grid_w, rope_split=cfg.rope_split,
+                              rope_base=cfg.rope_base, max_rounds=total_rounds),
+                  device=dev, page_order=wf_inputs.draw_page_order(npages, cfg.seed + 1))
+    shape = (cfg.num_slots, cfg.chunk_tokens, cfg.num_heads, cfg.head_dim)
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(cfg.seed * 1000 + rank)
+    inputs = []
+    for _ in range(2):   # two rounds of q, k, v, cycled
+        inputs.append([torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).to(tdt)
+                       for _ in range(3)])
+    if cfg.k_outlier_frac > 0:
+        for x in inputs:
+            m = torch.rand(shape[:3], generator=gen, device=dev) < cfg.k_outlier_frac
+            x[1] = torch.where(m[..., None], x[1].float() * cfg.k_outlier_scale, x[1].float()).to(tdt)
+    q_rot = torch.empty(shape, dtype=tdt, device=dev)
+    out = torch.empty(shape, dtype=tdt, device=dev)
+
+    def step(i):
+        x = inputs[i & 1]
+        pool.publish(0, x[0], x[1], x[2], q_rot)
+        pool.attention(0, q_rot, out)
+        pool.advance()
+
+    # pipeline fill (untimed, not counted as warm-up)
+    for i in range(steady):
+        step(i)
+    for i in range(args.warmup):
+        step(i)
+    st = pool.check_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    layout = pool.layout()
+    flops = unmasked_flops(layout, cfg)
+    pbytes = publish_bytes(layout, cfg)
+
+    import torch.distributed as dist
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    e_pub = [(ev(), ev()) for _ in range(args.steps)]
+    e_att = [(ev(), ev()) for _ in range(args.steps)]
+    t0, t1 = ev(), ev()
+    clocks = ClockSampler(local)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t0.record(stream)
+    for i in range(args.steps):
+        x = inputs[i & 1]
+        e_pub[i][0].record(stream)
+        pool.publish(0, x[0], x[1], x[2], q_rot)
+        e_pub[i][1].record(stream)
+        e_att[i][0].record(stream)
+        pool.attention(0, q_rot, out)
+        e_att[i][1].record(stream)
+        pool.advance()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if ws > 1:
+        dist.barrier()
+    st = pool.check_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timed steps")
+    ms = t0.elapsed_time(t1)
+    att_ms = statistics.mean(a.elapsed_time(b) for a, b in e_att)
+    pub_ms = statistics.mean(a.elapsed_time(b) for a, b in e_pub)
+    if ws > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    res = {"ms": ms, "att_ms": att_ms, "pub_ms": pub_ms, "flops": flops, "pbytes": pbytes,
+           "clocks": clk, "layout_positions": len(layout)}
+
+    # end to end: host buffers, H2D of the step's inputs, the C-ABI calls, D2H of out
+    if not args.no_e2e:
+        host_in = [[t.cpu().pin_memory() for t in x] for x in inputs]
+        host_out = torch.empty(shape, dtype=tdt).pin_memory()
+        dev_in = [torch.empty(shape, dtype=tdt, device=dev) for _ in range(3)]
+        h2d = sum(t.numel() * t.element_size() for t in host_in[0])
+        d2h = host_out.numel() * host_out.element_size()
+
+        def e2e_step(i):
+            for d, h in zip(dev_in, host_in[i & 1]):
+                d.copy_(h, non_blocking=True)
+            pool.publish(0, dev_in[0], dev_in[1], dev_in[2], q_rot)
+            pool.attention(0, q_rot, out)
+            pool.advance()
+            host_out.copy_(out, non_blocking=True)
+
+        e2e_step(0)
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+        a, b = ev(), ev()
+        a.record(stream)
+        for i in range(args.e2e_steps):
+            e2e_step(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        if ws > 1:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        res["e2e"] = {"ms": e_ms, "steps": args.e2e_steps, "h2d": h2d, "d2h": d2h}
+        st = pool.check_status()
+        if st != 0:
+            raise RuntimeError(f"device status {st} after e2e steps")
+    pool.close()
+    return res
+
+
+# ------------------------------------------------------------------- oracle timing
+
+def oracle_sample_rate(cfg, seconds, seed=0):
+    """Time the float64 oracle on a bounded sample of one steady round: the
+    same query rows of every live slot, one head, against each slot's full
+    visible context, rotary included. Returns (TFLOP/s, description)."""
+    import numpy as np
+    from oracle import wf_oracle as O
+    S, A, H = cfg.num_stages, cfg.anchor_chunks, cfg.history_chunks
+    lay = O.round_layout(S, A, H, cfg.steady_round())
+    rng = np.random.default_rng(seed)
+    C, d = cfg.chunk_tokens, cfg.head_dim
+
+    def rope(x, chunk):
+        if not cfg.rope:
+            return x
+        return O.rope_3d(x, chunk, cfg.frames_per_chunk, cfg.grid_h, cfg.grid_w,
+                         cfg.rope_split, cfg.rope_base)
+
+    keys = {p.chunk: rng.standard_normal((C, 1, d)) for p in lay}
+    vals = {p.chunk: rng.standard_normal((C, 1, d)) for p in lay}
+    q = rng.standard_normal((C, 1, d))
+
+    def once(rows):
+        kk = {c: rope(x, c) for c, x in keys.items()}
+        qr = {p.slot: rope(q, p.chunk) for p in lay if p.slot is not None}
+        O.attention_slot_prefix(qr, kk, vals, lay, rows=rows)
+        return _unmasked_rows_flops(lay, len(rows), C, d)
+
+    t0 = time.perf_counter()
+    once(np.arange(min(16, C)))
+    dt = time.perf_counter() - t0
+    n = int(max(16, min(C, 16 * (seconds / 4) / max(dt, 1e-4))))
+    rows = np.arange(n)
+    fl, reps = 0, 0
+    t0 = time.perf_counter()
+    while True:
+        fl += once(rows)
+        reps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    desc = (f"{reps} x ({len(rows)} query rows x 1 head of every live slot of a steady round, "
+            f"each against its full visible context, rotary included), {dt:.1f} s")
+    return fl / dt / 1e12, desc
+
+
+def _unmasked_rows_flops(lay, nrows, C, d):
+    tot = 0
+    for idx, p in enumerate(lay):
+        if p.slot is not None:
+            tot += 4 * nrows * (idx + 1) * C * d
+    return tot
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else None
+    except Exception:
+        return None
+
+
+def run_reference(args, ws, rank):
+    import wf_inputs
+    cfg = wf_inputs.CONFIGS[args.config]
+    if rank != 0:
+        return
+    per_step = max(0.5, min(4.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample_rate(cfg, per_step / 4)
+    rates = []
+    t0 = time.perf_counter()
+    descs = None
+    for _ in range(args.steps):
+        r, descs = oracle_sample_rate(cfg, per_step)
+        rates.append(r)
+    wall = time.perf_counter() - t0
+    v = statistics.mean(rates)
+    cores = len(os.sched_getaffinity(0))
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(cfg, args.gpus),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": blas_threads() or cores,
+                             "kind": "oracle", "sample": descs},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfg, n):
+    return {"workload": f"{cfg.name}: one layer-round, S={cfg.num_stages}+store, "
+                        f"C={cfg.chunk_tokens}, heads={cfg.num_heads}x{cfg.head_dim}, "
+                        f"anchor={cfg.anchor_chunks}, history={cfg.history_chunks}, "
+                        f"page={cfg.page_tokens}, steady state",
+            "step": "wf_publish_kv + wf_round_attention + wf_advance_round",
+            "l2": "working set > 126 MB L2 (pool 233 MB + q/k/v/q_rot/out 360 MB); no flush",
+            "parallelism": f"replicas x{n}" if n > 1 else "single GPU"}
+
+
+def main():
+    args = parse()
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.impl == "reference":
+        run_reference(args, ws, rank)
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    import wf_inputs
+    cfg = wf_inputs.CONFIGS[args.config]
+    res = run_ours(args, ws, rank, local)
+    if rank == 0:
+        peaks, src = read_peaks()
+        ms_step = res["ms"] / args.steps
+        value = ws * res["flops"] * args.steps / (res["ms"] * 1e-3) / 1e12
+        att_tflops = res["flops"] / (res["att_ms"] * 1e-3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        pub_gbs = res["pbytes"] / (res["pub_ms"] * 1e-3) / 1e9
+        kfile = os.path.join(ROOT, "chunk_causal_wavefront_b200", "csrc", "attn_bf16.cu")
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "config": workload_config(cfg, ws),
+            "rounds_per_s": ws * args.steps / (res["ms"] * 1e-3),
+            "attention": {"ms_per_launch": res["att_ms"], "tflops": att_tflops,
+                          "pct_bf16_peak_burst": 100 * att_tflops / peaks["bf16_tflops"],
+                          "pct_bf16_peak_sustained": 100 * att_tflops / peak,
+                          "flops_per_launch": res["flops"]},
+            "publish": {"ms_per_launch": res["pub_ms"], "gbs": pub_gbs,
+                        "pct_hbm": 100 * pub_gbs / peaks["hbm_gbs"],
+                        "bytes_per_launch": res["pbytes"]},
+            "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": peak,
+                         "unit": "TFLOP/s", "frac": att_tflops / peak,
+                         "traffic": read_traffic(kfile),
+                         "kernel": "attn_bf16_kernel",
+                         "peak_source": f"{src} bf16_tflops_sustained"},
+            "clocks": res["clocks"],
+            "gpu_launches": 3 * args.steps,
+        }
+        if "e2e" in res:
+            e = res["e2e"]
+            line["e2e"] = {"value": ws * res["flops"] * e["steps"] / (e["ms"] * 1e-3) / 1e12,
+                           "unit": UNIT, "h2d_bytes_per_step": e["h2d"],
+                           "d2h_bytes_per_step": e["d2h"], "steps": e["steps"]}
+        if ws == 1 and not args.no_cpu_baseline:
+            v, desc = oracle_sample_rate(cfg, args.cpu_seconds)
+            line["cpu_baseline"] = {"value": v, "unit": UNIT,
+                                    "cores": blas_threads() or len(os.sched_getaffinity(0)),
+                                    "kind": "oracle", "sample": desc}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

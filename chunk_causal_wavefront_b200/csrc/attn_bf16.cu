@@ -1,0 +1,401 @@
+// Round attention, bf16 tensor-core path for sm_100a (tcgen05 + TMEM + TMA).
+//
+// "Wave Forcing: Towards Speed-of-Light Streaming Video Generation", Method
+// section: full attention inside each chunk, chunk-wise causal attention across
+// chunks with M_WF(s, j) = 1[j >= s]; the ordered context of "Como funciona"
+// (anchor || history || store || denoising K/V) makes the keys of query slot s
+// a prefix of the context, so masked (s, j) chunk pairs are simply never
+// visited: the loop over key tiles stops at the slot's own chunk.
+//
+// One CTA computes O = softmax(Q K^T / sqrt(d)) V for one 128-row query tile
+// of one (slot, head) with the flash-attention online softmax:
+//   warp 4 (one lane)  TMA producer: Q once, then for every key tile (one
+//                      128-token page) K and V through the page table into a
+//                      two-stage shared-memory ring (128-byte swizzle);
+//   warp 5 (one lane)  tcgen05 issuer: S = Q K^T into one of two TMEM S
+//                      buffers (so S(j+1) overlaps the softmax of tile j), and
+//                      O += P V into a TMEM O accumulator;
+//   warps 0-3          softmax: thread r owns query row r (TMEM lane r); row
+//                      max and sum are thread-local over its 128 columns; P is
+//                      rounded to bf16 and written to shared memory in the
+//                      swizzled K-major layout the tensor core reads; O is
+//                      rescaled in TMEM only when the running max grows by more
+//                      than 2^8 (the exponentials stay <= 256 otherwise); the
+//                      epilogue divides by the row sum and stores bf16 rows.
+// Every wait is bounded: on timeout the CTA records WF_ERR_TIMEOUT, the other
+// roles see the abort flag, in-flight copies and MMAs are drained and TMEM is
+// freed before the CTA exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+#include "wf_internal.h"
+
+namespace wf {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;              // query rows per CTA
+constexpr int kBN = 128;              // keys per tile (one page)
+constexpr int kHD = 128;              // head dim
+constexpr uint32_t kHalf = 16384;     // one [128 rows][64 cols] bf16 swizzled block
+constexpr uint32_t kTile = 2 * kHalf; // [128][128] bf16
+constexpr int kPageCache = 1024;      // page ids cached in shared memory
+constexpr int kThreads = 192;
+constexpr long long kWaitLimit = 2000000000LL;  // ~1 s at 2 GHz
+
+// Shared-memory map (offsets from a 1024-byte aligned base).
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kOffQ + kTile;          // 2 stages
+constexpr uint32_t kOffV = kOffK + 2 * kTile;      // 2 stages
+constexpr uint32_t kOffP = kOffV + 2 * kTile;
+constexpr uint32_t kOffBar = kOffP + kTile;
+constexpr int kNumBars = 16;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr uint32_t kOffPages = kOffMisc + 64;
+constexpr uint32_t kSmemBytes = kOffPages + kPageCache * 4 + 1024;   // + alignment slack
+
+enum Bar {
+  kQFull = 0, kKFull0 = 1, kKEmpty0 = 3, kVFull0 = 5, kVEmpty0 = 7,
+  kSFull0 = 9, kSFree0 = 11, kPFull = 13, kPVDone = 14, kDrain = 15
+};
+
+struct Ctx {
+  uint64_t *bars;
+  volatile int *abort;
+  int32_t *status;
+};
+
+// Bounded wait on an mbarrier phase. Returns false (and flags the CTA) on
+// timeout or when another role has already aborted.
+__device__ __forceinline__ bool wait_bar(const Ctx &c, int b, uint32_t parity) {
+  uint64_t *bar = c.bars + b;
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 127u) == 0) {
+      if (*c.abort) return false;
+      if (clock64() - t0 > kWaitLimit) {
+        *c.abort = 1;
+        record_status(c.status, WF_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Time-bounded wait used while draining (ignores the abort flag).
+__device__ __forceinline__ void drain_wait(const Ctx &c, int b, uint32_t parity) {
+  uint64_t *bar = c.bars + b;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimit) {
+      record_status(c.status, WF_ERR_TIMEOUT);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Keep the compiler from using tcgen05.ld results before tcgen05.wait::ld.
+#define WF_REG_FENCE8(r, o)                                                                 \
+  asm volatile("" : "+r"(r[o + 0]), "+r"(r[o + 1]), "+r"(r[o + 2]), "+r"(r[o + 3]),         \
+               "+r"(r[o + 4]), "+r"(r[o + 5]), "+r"(r[o + 6]), "+r"(r[o + 7]))
+
+__device__ __forceinline__ void reg_fence32(uint32_t *r) {
+  WF_REG_FENCE8(r, 0);
+  WF_REG_FENCE8(r, 8);
+  WF_REG_FENCE8(r, 16);
+  WF_REG_FENCE8(r, 24);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bf16_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tq,
+                     const __grid_constant__ CUtensorMap tkv) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+  int32_t *page_cache = reinterpret_cast<int32_t *>(smem + kOffPages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // Work item: head-major; inside a head, slots in decreasing context length
+  // (slot 0 first: longest first), then query tiles.
+  const int tiles = (p.C + kBM - 1) / kBM;
+  const int per_head = p.live.n * tiles;
+  const int h = blockIdx.x / per_head;
+  const int rem = blockIdx.x - h * per_head;
+  const int li = p.live.n - 1 - rem / tiles;
+  const int tile = rem % tiles;
+  const int slot = p.live.slot[li];
+  const int npos = p.live.npos[li];
+  const int row0 = tile * kBM;
+
+  // Readiness + bounds check of the whole round's context (so that a stale
+  // page stops every CTA of the launch), caching this item's page ids.
+  {
+    int bad = 0, stale = 0;
+    const int total = p.n_pos * p.npc;
+    for (int i = threadIdx.x; i < total; i += blockDim.x) {
+      const int pos = i / p.npc;
+      const int pg = __ldcg(p.table + kTabPages + i);
+      if (pg < 0 || pg >= p.num_pages) bad = 1;
+      else if (__ldcg(p.tags + pg) != __ldcg(p.table + kTabPosTag + pos)) stale = 1;
+      if (i < kPageCache) page_cache[i] = pg;
+    }
+    if (threadIdx.x == 0) {
+      *abort_flag = 0;
+      for (int b = 0; b < kNumBars; ++b) {
+        const bool softmax_arrives = b == kSFree0 || b == kSFree0 + 1 || b == kPFull;
+        mbar_init(bars + b, softmax_arrives ? kBM : 1);
+      }
+      fence_barrier_init();
+    }
+    const int any_bad = __syncthreads_or(bad);
+    const int any_stale = __syncthreads_or(stale);
+    if (any_bad || any_stale) {
+      if (threadIdx.x == 0) record_status(p.status, any_bad ? WF_ERR_BAD_PAGE : WF_ERR_NOT_READY);
+      return;
+    }
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Ctx ctx{bars, abort_flag, p.status};
+  const int n_tiles = npos * p.npc;
+  const int last_valid = p.C - (p.npc - 1) * p.P;   // keys in a chunk's last page
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      tma_prefetch_desc(&tq);
+      tma_prefetch_desc(&tkv);
+      uint8_t *sQ = smem + kOffQ;
+      mbar_arrive_expect_tx(bars + kQFull, kTile);
+      tma_load_4d(sQ, &tq, bars + kQFull, 0, h, row0, slot);
+      tma_load_4d(sQ + kHalf, &tq, bars + kQFull, 64, h, row0, slot);
+      int nk[2] = {0, 0}, nv[2] = {0, 0};
+      for (int j = 0; j < n_tiles; ++j) {
+        const int stg = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        const int idx = j;   // (position, page) flattened == tile index
+        const int phys = idx < kPageCache ? page_cache[idx] : __ldcg(p.table + kTabPages + idx);
+        const int rowk = static_cast<int>(p.layer_row0) + ((phys * 2) * p.Hh + h) * p.P;
+        const int rowv = rowk + p.Hh * p.P;
+        uint8_t *sK = smem + kOffK + stg * kTile;
+        uint8_t *sV = smem + kOffV + stg * kTile;
+        if (!wait_bar(ctx, kKEmpty0 + stg, ph ^ 1)) break;
+        mbar_arrive_expect_tx(bars + kKFull0 + stg, kTile);
+        tma_load_2d(sK, &tkv, bars + kKFull0 + stg, 0, rowk);
+        tma_load_2d(sK + kHalf, &tkv, bars + kKFull0 + stg, 64, rowk);
+        ++nk[stg];
+        if (!wait_bar(ctx, kVEmpty0 + stg, ph ^ 1)) break;
+        mbar_arrive_expect_tx(bars + kVFull0 + stg, kTile);
+        tma_load_2d(sV, &tkv, bars + kVFull0 + stg, 0, rowv);
+        tma_load_2d(sV + kHalf, &tkv, bars + kVFull0 + stg, 64, rowv);
+        ++nv[stg];
+      }
+      // Drain: every load this thread issued has landed before the CTA exits.
+      for (int s = 0; s < 2; ++s) {
+        if (nk[s]) drain_wait(ctx, kKFull0 + s, (nk[s] - 1) & 1);
+        if (nv[s]) drain_wait(ctx, kVFull0 + s, (nv[s] - 1) & 1);
+      }
+      drain_wait(ctx, kQFull, 0);
+    }
+  } else if (warp == 5) {
+    // ---------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t idS = make_idesc_bf16(kBM, kBN, false);
+      constexpr uint32_t idPV = make_idesc_bf16(kBM, kHD, true);
+      const uint32_t tO = tmem + 256;
+      const uint32_t aQ = smem_u32(smem + kOffQ);
+      const uint32_t aP = smem_u32(smem + kOffP);
+      bool ok = wait_bar(ctx, kQFull, 0);
+      tc_fence_after();
+      auto issue_s = [&](int j) -> bool {
+        const int stg = j & 1, b = j & 1;
+        if (!wait_bar(ctx, kKFull0 + stg, (j >> 1) & 1)) return false;
+        if (j >= 2 && !wait_bar(ctx, kSFree0 + b, ((j - 2) >> 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t aK = smem_u32(smem + kOffK + stg * kTile);
+#pragma unroll
+        for (int k = 0; k < kHD / 16; ++k) {
+          const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
+          mma_bf16_ss(tmem + b * 128, make_desc_sw128(aQ + off, 16, 1024),
+                      make_desc_sw128(aK + off, 16, 1024), idS, k > 0);
+        }
+        mma_commit(bars + kSFull0 + b);
+        mma_commit(bars + kKEmpty0 + stg);
+        return true;
+      };
+      if (ok && n_tiles > 0) ok = issue_s(0);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        if (j + 1 < n_tiles && !issue_s(j + 1)) break;
+        const int stg = j & 1;
+        if (!wait_bar(ctx, kPFull, j & 1)) break;
+        if (!wait_bar(ctx, kVFull0 + stg, (j >> 1) & 1)) break;
+        tc_fence_after();
+        const uint32_t aV = smem_u32(smem + kOffV + stg * kTile);
+#pragma unroll
+        for (int k = 0; k < kBN / 16; ++k) {
+          const uint64_t da = make_desc_sw128(aP + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
+          const uint64_t db = make_desc_sw128(aV + k * 2048, kHalf, 1024);
+          mma_bf16_ss(tO, da, db, idPV, (j > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(bars + kVEmpty0 + stg);
+        mma_commit(bars + kPVDone);
+      }
+      // Drain: all MMAs issued by this thread complete before TMEM is freed.
+      mma_commit(bars + kDrain);
+      drain_wait(ctx, kDrain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------- softmax --
+    const int r = warp * 32 + lane;                     // query row == TMEM lane
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    uint8_t *sP = smem + kOffP;
+    float m = -INFINITY, l = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int b = j & 1;
+      ok = __all_sync(0xffffffffu, wait_bar(ctx, kSFull0 + b, (j >> 1) & 1));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_addr + b * 128 + c * 32, s + c * 32);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence32(s + c * 32);
+      tc_fence_before();
+      mbar_arrive(bars + kSFree0 + b);
+
+      const int valid = (j % p.npc == p.npc - 1) ? last_valid : kBN;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        if (c >= valid) s[c] = __float_as_uint(-INFINITY);
+        mx = fmaxf(mx, __uint_as_float(s[c]));
+      }
+      const float m_new = fmaxf(m, mx * p.scale_log2);
+      const bool rescale = (j == 0) || (m_new - m > 8.0f);
+      const float alpha = rescale ? ex2(m - m_new) : 1.0f;
+      const float m_use = rescale ? m_new : m;
+      float rowsum = 0.0f;
+      uint32_t pw[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = ex2(fmaf(__uint_as_float(s[2 * c]), p.scale_log2, -m_use));
+        const float p1 = ex2(fmaf(__uint_as_float(s[2 * c + 1]), p.scale_log2, -m_use));
+        __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+        pw[c] = *reinterpret_cast<uint32_t *>(&pb);
+        rowsum += __uint_as_float(pw[c] << 16) + __uint_as_float(pw[c] & 0xFFFF0000u);
+      }
+      l = l * alpha + rowsum;
+      m = m_use;
+
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, wait_bar(ctx, kPVDone, (j - 1) & 1));
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_addr + 256 + c * 32, o);
+            tmem_ld_wait();
+            reg_fence32(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tmem + lane_addr + 256 + c * 32, o);
+          }
+          tmem_st_wait();
+        }
+      }
+      // P row -> shared memory, K-major with the 128-byte swizzle: 16-byte
+      // chunk c of row r in 64-key half kt lands at r*128 + ((c ^ (r & 7)) * 16).
+#pragma unroll
+      for (int cc = 0; cc < 16; ++cc) {
+        const int kt = cc >> 3, c = cc & 7;
+        const uint32_t addr = smem_u32(sP + kt * kHalf + r * 128 + ((c ^ (r & 7)) << 4));
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pw[4 * cc]),
+                     "r"(pw[4 * cc + 1]), "r"(pw[4 * cc + 2]), "r"(pw[4 * cc + 3])
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bars + kPFull);
+    }
+    if (ok && n_tiles > 0) {
+      ok = __all_sync(0xffffffffu, wait_bar(ctx, kPVDone, (n_tiles - 1) & 1));
+    }
+    if (ok && n_tiles > 0) {
+      tc_fence_after();
+      const float inv = 1.0f / l;
+      const int n = row0 + r;
+      __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) +
+                           ((static_cast<size_t>(slot) * p.C + n) * p.Hh + h) * kHD;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_addr + 256 + c * 32, o);
+        tmem_ld_wait();
+        reg_fence32(o);
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv,
+                                                   __uint_as_float(o[2 * i + 1]) * inv);
+          w[i] = *reinterpret_cast<uint32_t *>(&v);
+        }
+        if (n < p.C) {
+          uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attention_bf16(const AttnParams &p, const void *tmap_q, const void *tmap_kv,
+                                  cudaStream_t st) {
+  if (p.live.n == 0) return cudaSuccess;
+  if (p.d != kHD || p.P != kBN) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  const int tiles = (p.C + kBM - 1) / kBM;
+  const int64_t blocks = static_cast<int64_t>(tiles) * p.live.n * p.Hh;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  attn_bf16_kernel<<<static_cast<unsigned>(blocks), kThreads, kSmemBytes, st>>>(
+      p, *static_cast<const CUtensorMap *>(tmap_q), *static_cast<const CUtensorMap *>(tmap_kv));
+  return cudaGetLastError();
+}
+
+}  // namespace wf

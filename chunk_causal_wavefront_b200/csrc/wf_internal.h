@@ -1,0 +1,108 @@
+// Internal declarations shared by the libwf sources (host pool + kernels).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "wf.h"
+
+namespace wf {
+
+constexpr int kMaxSlots = WF_MAX_STAGES + 1;
+constexpr int kMaxPositions = 1 + WF_MAX_HISTORY + WF_MAX_STAGES + 1;
+
+// Device page table, rewritten (stream-ordered) on every round advance.
+// int32 words at these offsets inside the table region of the pool memory:
+//   [kTabRound]               round k
+//   [kTabNumPos]              number of positions in the ordered context
+//   [kTabSlotPos + s]         position index of slot s (store = S), -1 if idle
+//   [kTabSlotChunk + s]       chunk index held by slot s, -1 if idle
+//   [kTabPosTag + p]          ready tag expected for every page of position p
+//   [kTabPosChunk + p]        chunk index of position p
+//   [kTabPages + p*npc + j]   physical page of the j-th page of position p
+constexpr int kTabRound = 0;
+constexpr int kTabNumPos = 1;
+constexpr int kTabSlotPos = 2;
+constexpr int kTabSlotChunk = kTabSlotPos + kMaxSlots;
+constexpr int kTabPosTag = kTabSlotChunk + kMaxSlots;
+constexpr int kTabPosChunk = kTabPosTag + kMaxPositions;
+constexpr int kTabPages = kTabPosChunk + kMaxPositions;
+
+// Work description of one launch, built on the host from the host mirror.
+struct LiveSlots {
+  int32_t n;                       // live query slots this round
+  int32_t slot[kMaxSlots];         // slot ids (store = S)
+  int32_t chunk[kMaxSlots];        // chunk each holds
+  int32_t tag[kMaxSlots];          // ready tag its publish writes
+  int32_t npos[kMaxSlots];         // context prefix length it reads
+};
+
+struct PublishParams {
+  const void *q, *k, *v;
+  void *q_rot;
+  char *pages;                // this layer's page region
+  int32_t *tags;              // this layer's ready tags [num_pages]
+  const int32_t *table;       // device page table
+  int32_t *status;            // sticky status word
+  const float2 *rope_t, *rope_h, *rope_w;  // (cos, sin) per position x pair
+  int32_t S1, C, Hh, d, P, npc, num_pages;
+  int32_t rope, F, gh, gw, split0, split1, split2;
+  LiveSlots live;
+};
+
+struct AttnParams {
+  const void *q_rot;
+  void *out;
+  const char *pages;          // this layer's page region
+  const int32_t *tags;        // this layer's ready tags
+  const int32_t *table;
+  int32_t *status;
+  int32_t S1, C, Hh, d, P, npc, num_pages, n_pos;
+  int64_t layer_row0;         // first pool row of this layer (bf16 tensor map)
+  float scale_log2;           // log2(e) / sqrt(d)
+  float scale;                // 1 / sqrt(d)
+  LiveSlots live;
+};
+
+// Launchers (return a cudaError_t from the launch).
+cudaError_t launch_publish_bf16(const PublishParams &p, cudaStream_t st);
+cudaError_t launch_publish_f32(const PublishParams &p, cudaStream_t st);
+cudaError_t launch_attention_f32(const AttnParams &p, cudaStream_t st);
+// The bf16 tensor-core path takes the encoded tensor maps (opaque 128-byte
+// CUtensorMap objects) of q_rot, out and the pool's K/V pages.
+cudaError_t launch_attention_bf16(const AttnParams &p, const void *tmap_q,
+                                  const void *tmap_kv, cudaStream_t st);
+cudaError_t launch_table_upload(int32_t *dst, const int32_t *src, int n_words,
+                                cudaStream_t st);
+cudaError_t launch_poke(int32_t *dst, int32_t value, cudaStream_t st);
+
+#ifdef __CUDACC__
+// Record the first device-side error in the sticky status word.
+__device__ __forceinline__ void record_status(int32_t *status, int32_t code) {
+  atomicCAS(status, 0, code);
+}
+
+// Readiness and bounds check of every page in context positions [0, n_pos):
+// returns WF_OK, WF_ERR_BAD_PAGE or WF_ERR_NOT_READY (block-uniform).
+// Every thread of the block must call it.
+__device__ __forceinline__ int check_context_pages(const int32_t *table, const int32_t *tags,
+                                                   int n_pos, int npc, int num_pages) {
+  int bad_page = 0, stale = 0;
+  const int total = n_pos * npc;
+  for (int i = threadIdx.x; i < total; i += blockDim.x) {
+    const int p = i / npc;
+    const int pg = __ldcg(table + kTabPages + i);
+    if (pg < 0 || pg >= num_pages) {
+      bad_page = 1;
+    } else if (__ldcg(tags + pg) != __ldcg(table + kTabPosTag + p)) {
+      stale = 1;
+    }
+  }
+  if (__syncthreads_or(bad_page)) return WF_ERR_BAD_PAGE;
+  if (__syncthreads_or(stale)) return WF_ERR_NOT_READY;
+  return WF_OK;
+}
+#endif
+
+}  // namespace wf

@@ -1,0 +1,190 @@
+/*
+ * wf.h - C ABI of libwf: one causal-wavefront round of chunk-wise causal
+ * attention (Wave Forcing), on one NVIDIA B200 (sm_100a).
+ *
+ * Source: "Wave Forcing: Towards Speed-of-Light Streaming Video Generation"
+ * (arXiv 2611.00859). The method, as the pages state it:
+ *   - Method section (hyper.ai summary): a stage-s update of chunk i runs in
+ *     round k = i + s; full attention inside each chunk, chunk-wise causal
+ *     attention across chunks, mask M_WF(s, j) = 1[j >= s] (query slot s reads
+ *     itself and every cleaner slot j, never a noisier one); K/V are published
+ *     right after the QKV projection and RoPE, readiness is checked just before
+ *     attention, and paged delivery writes K/V straight into ordered attention
+ *     slots followed by a ready signal.
+ *   - "Como funciona" (e-cogni article): the ordered context of a layer is
+ *     anchor (initial chunk) || bounded clean history || live store ||
+ *     denoising K/V.
+ *   - Appendix Table 3: stages 0 <= s < S, the store is stage S; B_i = Z_i(S).
+ *
+ * Conventions for every call:
+ *   - Pointers named q, k, v, q_rot, out and dev_mem are DEVICE pointers on the
+ *     current CUDA device; config structs and page_order are HOST pointers.
+ *   - Activations are laid out [S+1][C][num_heads][head_dim], row-major, in the
+ *     pool's dtype (bf16 or fp32): slot-major, then token, head, dimension.
+ *     Slot s < S holds the chunk at denoising stage s; slot S is the store.
+ *   - Every call that takes a stream enqueues its device work on that stream
+ *     (NULL = legacy default stream) and returns without synchronising, except
+ *     wf_kv_pool_create (synchronises once, at set-up) and
+ *     wf_pool_check_status. No call allocates device memory.
+ *   - Errors found on the host return at once and enqueue nothing. Errors found
+ *     by a kernel (a slot read before it was published, a page id out of range)
+ *     are recorded in a sticky status word inside the pool memory; the kernel
+ *     that found them writes no output, and the next wf_pool_check_status
+ *     returns (and clears) the first one recorded.
+ *   - A pool is not thread-safe; calls on one pool must be issued in program
+ *     order on one stream (or streams ordered by the caller).
+ */
+#ifndef WF_H_
+#define WF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *wf_stream_t;
+
+typedef enum {
+  WF_OK = 0,
+  WF_ERR_INVALID_ARG = 1,   /* bad config, pointer, size, layer or alignment */
+  WF_ERR_OUT_OF_PAGES = 2,  /* num_pages below the minimum the schedule needs */
+  WF_ERR_NOT_READY = 3,     /* attention found a page whose ready tag is stale */
+  WF_ERR_BAD_PAGE = 4,      /* a page-table entry points outside the pool */
+  WF_ERR_CALL_ORDER = 5,    /* call not allowed in the pool's current state */
+  WF_ERR_CUDA = 6,          /* a CUDA runtime/driver call failed */
+  WF_ERR_UNSUPPORTED = 7,   /* valid but not implemented shape/dtype combo */
+  WF_ERR_TIMEOUT = 8        /* a bounded device-side wait ran out (kernel gave up) */
+} wf_status;
+
+enum { WF_DTYPE_BF16 = 0, WF_DTYPE_F32 = 1 };
+enum { WF_ROPE_OFF = 0, WF_ROPE_3D = 1 };
+
+/* Limits of this implementation. */
+#define WF_MAX_STAGES 16
+#define WF_MAX_HISTORY 64
+
+typedef struct {
+  int32_t num_stages;      /* S, 1..WF_MAX_STAGES; slots 0..S-1 plus the store */
+  int32_t chunk_tokens;    /* C, tokens per chunk (full attention inside) */
+  int32_t num_heads;       /* attention heads (K/V heads = Q heads) */
+  int32_t head_dim;        /* d; bf16 attention: 128; fp32: multiple of 4, <= 128 */
+  int32_t anchor_chunks;   /* 0 or 1: keep chunk 0 as the anchor */
+  int32_t history_chunks;  /* H, bounded clean history window, 0..WF_MAX_HISTORY */
+  int32_t page_tokens;     /* P, tokens per page; bf16 attention: 128 */
+  int32_t num_layers;      /* layers sharing the page table (one pool region each) */
+  int32_t dtype;           /* WF_DTYPE_BF16 or WF_DTYPE_F32 */
+  int32_t rope;            /* WF_ROPE_OFF or WF_ROPE_3D */
+  int32_t frames_per_chunk;/* F: latent frames per chunk (3D rotary only) */
+  int32_t grid_h, grid_w;  /* patch grid per frame; C == F * grid_h * grid_w */
+  int32_t rope_split[3];   /* rotary band widths over t, h, w; even, sum = d */
+  float rope_base;         /* rotary base (10000) */
+  int32_t max_rounds;      /* rounds the pool may run (sizes the t table) */
+  int32_t num_pages;       /* physical pages per layer; 0 = the minimum */
+} wf_pool_config;
+
+typedef struct wf_pool wf_pool;
+
+/* Where things live inside the caller's pool memory (for tests and tools). */
+typedef struct {
+  int64_t num_pages;        /* physical pages per layer */
+  int32_t pages_per_chunk;  /* ceil(C / P) */
+  int32_t max_positions;    /* A + H + S + 1 */
+  size_t status_offset;     /* int32 sticky status word */
+  size_t tags_offset;       /* int32 [num_layers][num_pages] ready tags */
+  size_t pages_offset;      /* [num_layers][num_pages][2 (K,V)][heads][P][d] */
+  size_t page_bytes;        /* bytes of one (layer, page): 2 * heads * P * d * elt */
+  size_t total_bytes;       /* == wf_kv_pool_bytes */
+} wf_pool_geometry;
+
+/* Bytes of device memory a pool with this config needs (the caller allocates
+ * them, 256-byte aligned, and keeps them alive until wf_pool_destroy).
+ * Returns WF_ERR_INVALID_ARG / WF_ERR_OUT_OF_PAGES / WF_ERR_UNSUPPORTED for a
+ * config that wf_kv_pool_create would reject. */
+wf_status wf_kv_pool_bytes(const wf_pool_config *cfg, size_t *bytes);
+
+/* Create the paged K/V pool: page table, free list, ordered slots, ready tags
+ * (paged delivery into ordered attention slots, Method section; the bounded
+ * history window of "Como funciona").
+ *   dev_mem, bytes : caller-owned device memory of wf_kv_pool_bytes bytes,
+ *                    256-byte aligned; NULL/0 creates a host-only pool that
+ *                    runs the bookkeeping (advance, layout queries) with no
+ *                    device work, for dry runs and CPU tests.
+ *   page_order     : host array of num_pages distinct ids in [0, num_pages)
+ *                    giving the initial free-list order, or NULL (identity).
+ *   stream         : stream for the set-up writes; the call synchronises it.
+ * On success *out owns the host state; the pool starts at round 0. */
+wf_status wf_kv_pool_create(const wf_pool_config *cfg, void *dev_mem, size_t bytes,
+                            const int32_t *page_order, wf_stream_t stream, wf_pool **out);
+
+/* Publish one layer's K/V for every live slot of the current round (early
+ * publication after QKV + RoPE, Method section): applies the 3D rotary
+ * embedding to q and k (fp32 math, one rounding), writes q_rot, scatters
+ * rotated K and V into the slots' pages (rows past C in a chunk's last page
+ * are zeroed) and stamps each written page's ready tag.
+ *   q, k, v : inputs, [S+1][C][heads][d]; rows of slots that are not live in
+ *             this round are not read.
+ *   q_rot   : output, same layout; only live slots' rows are written.
+ * Pointers must be 16-byte aligned; q_rot must not alias q, k or v. */
+wf_status wf_publish_kv(wf_pool *pool, int32_t layer, const void *q, const void *k,
+                        const void *v, void *q_rot, wf_stream_t stream);
+
+/* Round attention for one layer (M_WF mask, full attention inside chunks):
+ * for every live query slot s and head h,
+ *     out[s] = softmax(q_rot[s] K_s^T / sqrt(d)) V_s
+ * where K_s, V_s are the keys of the ordered-context prefix slot s may read
+ * (anchor, history, store, slots S-1 .. s). Before reading, the kernel checks
+ * every page's ready tag against the round's expected tag; any mismatch sets
+ * WF_ERR_NOT_READY in the status word and the launch writes no output.
+ *   q_rot : [S+1][C][heads][d] rotated queries (as written by wf_publish_kv);
+ *   out   : [S+1][C][heads][d]; rows of non-live slots are left untouched.
+ * bf16 pools need head_dim == 128 and page_tokens == 128 (tensor-core path);
+ * fp32 pools run a CUDA-core path. Pointers must be 16-byte aligned. */
+wf_status wf_round_attention(wf_pool *pool, int32_t layer, const void *q_rot, void *out,
+                             wf_stream_t stream);
+
+/* Move the pool to the next round (k -> k + 1, Table 3): the store's chunk
+ * becomes the anchor (chunk 0, when kept) or the newest history chunk; history
+ * beyond H returns its pages to the free list; the next store takes pages
+ * from the free list; the device page table is rewritten on the stream.
+ * Returns WF_ERR_CALL_ORDER when max_rounds would be exceeded. */
+wf_status wf_advance_round(wf_pool *pool, wf_stream_t stream);
+
+/* Synchronise the stream, then return and clear the pool's sticky device
+ * status (WF_OK if no kernel recorded an error). */
+wf_status wf_pool_check_status(wf_pool *pool, wf_stream_t stream);
+
+/* Free the host state. Does not touch dev_mem (the caller owns it). */
+wf_status wf_pool_destroy(wf_pool *pool);
+
+const char *wf_status_string(wf_status status);
+
+/* Current round k, or -1 for a NULL pool. */
+int64_t wf_pool_round(const wf_pool *pool);
+
+/* Region offsets inside dev_mem. */
+wf_status wf_pool_get_geometry(const wf_pool *pool, wf_pool_geometry *geom);
+
+/* The current round's ordered context, from the host mirror of the page table.
+ * Writes *n_positions and, for each position p < cap: kinds[p] (0 anchor,
+ * 1 history, 2 store, 3 denoising slot), chunks[p], slots[p] (-1 for anchor
+ * and history), tags[p] (expected ready tag) and
+ * pages[p * pages_per_chunk + j] (physical page of the chunk's j-th page).
+ * Any output pointer may be NULL. */
+wf_status wf_pool_get_layout(const wf_pool *pool, int32_t *n_positions, int32_t *kinds,
+                             int32_t *chunks, int32_t *slots, int32_t *tags,
+                             int32_t *pages, int32_t cap);
+
+/* Fault-injection hook for tests: overwrite one entry of the DEVICE page table
+ * (position, j) with `physical` (which may be out of range), without changing
+ * the host mirror. The next publish/attention sees it; kernels bounds-check
+ * page ids and record WF_ERR_BAD_PAGE instead of accessing memory. */
+wf_status wf_pool_debug_poke_page(wf_pool *pool, int32_t position, int32_t j,
+                                  int32_t physical, wf_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WF_H_ */

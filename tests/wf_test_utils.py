@@ -1,0 +1,162 @@
+"""Helpers that drive libwf and the float64 oracle side by side.
+
+Inputs come from wf_inputs (seeded, rounded once to the working dtype); the
+oracle side widens exactly those bits to float64 and applies its own rotary
+embedding and attention. Nothing here computes the method on the GPU side: the
+library does, through its C ABI.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+import torch
+
+import wf_inputs
+from wf_inputs import WorkloadConfig, bf16_bits_to_f64
+from oracle import wf_oracle as O
+
+
+def pool_config(cfg: WorkloadConfig, **over):
+    from chunk_causal_wavefront_b200 import make_config
+    kw = dict(num_stages=cfg.num_stages, chunk_tokens=cfg.chunk_tokens, num_heads=cfg.num_heads,
+              head_dim=cfg.head_dim, anchor_chunks=cfg.anchor_chunks,
+              history_chunks=cfg.history_chunks, page_tokens=cfg.page_tokens,
+              num_layers=cfg.num_layers, dtype=cfg.dtype, rope=cfg.rope,
+              frames_per_chunk=cfg.frames_per_chunk, grid_h=cfg.grid_h, grid_w=cfg.grid_w,
+              rope_split=cfg.rope_split if cfg.rope else (0, 0, 0), rope_base=cfg.rope_base,
+              max_rounds=max(cfg.rounds + 1, 16), num_pages=0)
+    kw.update(over)
+    return make_config(**kw)
+
+
+def min_pages(cfg: WorkloadConfig) -> int:
+    return (cfg.num_stages + 1 + cfg.anchor_chunks + cfg.history_chunks) * cfg.pages_per_chunk
+
+
+def to_f64(arr: np.ndarray, dtype: str) -> np.ndarray:
+    return bf16_bits_to_f64(arr) if dtype == "bf16" else arr.astype(np.float64)
+
+
+def to_device(arr: np.ndarray, dtype: str, device) -> torch.Tensor:
+    if dtype == "bf16":
+        return torch.from_numpy(arr.view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(arr).to(device)
+
+
+def tensor_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().double().numpy()
+
+
+def rel_l2(a: np.ndarray, b: np.ndarray) -> float:
+    return float(np.linalg.norm((a - b).ravel()) / max(np.linalg.norm(b.ravel()), 1e-300))
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 numbers at |x| (8 significant bits)."""
+    ax = np.maximum(np.abs(x), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(ax)) - 7)
+
+
+class Rollout:
+    """One pool on one GPU plus the oracle's view of the same rounds."""
+
+    def __init__(self, cfg: WorkloadConfig, device="cuda", page_seed: Optional[int] = 7,
+                 num_pages: int = 0, layers: Optional[int] = None):
+        from chunk_causal_wavefront_b200 import KVPool
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.layers = cfg.num_layers if layers is None else layers
+        n_pages = num_pages or min_pages(cfg)
+        self.page_order = (None if page_seed is None
+                           else wf_inputs.draw_page_order(n_pages, page_seed))
+        self.pool = KVPool(pool_config(cfg, num_layers=self.layers, num_pages=num_pages),
+                           device=self.device, page_order=self.page_order)
+        shape = (cfg.num_slots, cfg.chunk_tokens, cfg.num_heads, cfg.head_dim)
+        tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+        self.q_rot = torch.zeros(shape, dtype=tdt, device=self.device)
+        self.out = torch.zeros(shape, dtype=tdt, device=self.device)
+        self.stored: Dict[int, tuple] = {}   # chunk -> (k bits, v bits) the store published
+        self.live: Dict[int, tuple] = {}     # slot -> (q, k, v bits, chunk) this round
+
+    @property
+    def round(self) -> int:
+        return self.pool.round
+
+    def layout(self):
+        c = self.cfg
+        return O.round_layout(c.num_stages, c.anchor_chunks, c.history_chunks, self.round)
+
+    def publish(self, layer: int = 0, inputs=None, real_slots: Optional[Sequence[int]] = None):
+        """Draw (or take) this round's inputs and run wf_publish_kv."""
+        c = self.cfg
+        lay = self.layout()
+        live = [p.slot for p in lay if p.slot is not None]
+        if inputs is None:
+            slots = live if real_slots is None else [s for s in live if s in real_slots]
+            inputs = wf_inputs.draw_round_inputs(c, self.round, layer, slots=slots)
+        q, k, v = inputs
+        self.inputs = inputs
+        tq, tk, tv = (to_device(x, c.dtype, self.device) for x in (q, k, v))
+        self.pool.publish(layer, tq, tk, tv, self.q_rot)
+        self.live = {}
+        for p in lay:
+            if p.slot is None:
+                continue
+            self.live[p.slot] = (q[p.slot], k[p.slot], v[p.slot], p.chunk)
+            if p.kind == "store":
+                self.stored[p.chunk] = (k[p.slot], v[p.slot])
+        return inputs
+
+    def attention(self, layer: int = 0, fill: float = float("nan")):
+        self.out.fill_(fill)
+        self.pool.attention(layer, self.q_rot, self.out)
+
+    def advance(self):
+        self.pool.advance()
+
+    # ---- oracle side ----------------------------------------------------------------
+    def _rope(self, x64: np.ndarray, chunk: int) -> np.ndarray:
+        c = self.cfg
+        if not c.rope:
+            return x64
+        return O.rope_3d(x64, chunk, c.frames_per_chunk, c.grid_h, c.grid_w,
+                         split=c.rope_split, base=c.rope_base)
+
+    def oracle_tensors(self, heads: Sequence[int]):
+        """fp64 rotated q per live slot, rotated K and V per context chunk."""
+        c, hs = self.cfg, list(heads)
+        q_rot, keys, vals = {}, {}, {}
+        for s, (q, k, v, chunk) in self.live.items():
+            q_rot[s] = self._rope(to_f64(q, c.dtype)[:, hs], chunk)
+        for p in self.layout():
+            if p.slot is None:
+                kb, vb = self.stored[p.chunk]
+            else:
+                _, kb, vb, _ = self.live[p.slot]
+            keys[p.chunk] = self._rope(to_f64(kb, c.dtype)[:, hs], p.chunk)
+            vals[p.chunk] = to_f64(vb, c.dtype)[:, hs]
+        return q_rot, keys, vals
+
+    def oracle_out(self, heads: Sequence[int], rows: Optional[np.ndarray] = None):
+        q_rot, keys, vals = self.oracle_tensors(heads)
+        return O.attention_slot_prefix(q_rot, keys, vals, self.layout(), rows=rows)
+
+    def oracle_out_from_gpu_operands(self, heads: Sequence[int], rows=None):
+        """Oracle attention fed the GPU's own rounded q_rot and K/V pages."""
+        c, hs = self.cfg, list(heads)
+        pages = self.pool.pages_view()
+        qr = tensor_f64(self.q_rot)
+        q_rot, keys, vals = {}, {}, {}
+        for s in self.live:
+            q_rot[s] = qr[s][:, hs]
+        for kind, chunk, slot, tag, pgs in self.pool.layout():
+            kp = tensor_f64(pages[0, pgs, 0][:, hs])   # [npc][heads][P][d]
+            vp = tensor_f64(pages[0, pgs, 1][:, hs])
+            keys[chunk] = np.transpose(kp, (0, 2, 1, 3)).reshape(-1, len(hs), c.head_dim)[:c.chunk_tokens]
+            vals[chunk] = np.transpose(vp, (0, 2, 1, 3)).reshape(-1, len(hs), c.head_dim)[:c.chunk_tokens]
+        return O.attention_slot_prefix(q_rot, keys, vals, self.layout(), rows=rows)
+
+    def close(self):
+        self.pool.close()
