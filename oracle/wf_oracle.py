@@ -53,7 +53,7 @@ import numpy as np
 __all__ = [
     "Position", "round_layout", "visible_positions", "rope_positions", "rope_3d",
     "attention_slot_prefix", "attention_dense_mask", "attention_bruteforce",
-    "PoolModel", "expected_tag", "publish_pages", "unmasked_flops",
+    "PoolModel", "expected_tag", "publish_pages", "unmasked_flops", "round_bf16",
 ]
 
 
@@ -152,6 +152,29 @@ def rope_3d(x: np.ndarray, chunk: int, F: int, gh: int, gw: int,
         out[:, :, off:off + da:2] = a * c - b * s
         out[:, :, off + 1:off + da:2] = a * s + b * c
         off += da
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Storage format of published K/V.
+# ---------------------------------------------------------------------------
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 (8 significant bits, ties
+    to even), returned as float64.
+
+    The pages run the model in BF16 (Table 1's BF16/FA3 backend), so published
+    rotated queries and keys are bf16 values; this models that storage format.
+    Written from the definition: scale each value so its 8 significant bits are
+    the integer part, round half to even, scale back. Normal range only (the
+    inputs here are O(1)); zeros stay zero.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros_like(x)
+    nz = x != 0
+    e = np.floor(np.log2(np.abs(x[nz])))
+    scale = np.exp2(7.0 - e)
+    out[nz] = np.rint(x[nz] * scale) / scale          # np.rint rounds half to even
     return out
 
 

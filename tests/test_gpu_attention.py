@@ -1,11 +1,14 @@
 """GPU parity of wf_round_attention against the float64 oracle.
 
 Tolerances: fp32 max-abs 1e-5; bf16 max-abs 2e-2 and relative L2 1e-2, against
-the oracle fed the exact inputs (and, separately, fed the GPU's own rounded
-q_rot and K/V pages, which isolates the attention kernel's error from rotary
-rounding). Small cases cover every round of fill and steady state with
+the oracle fed the exact inputs and, separately, against the oracle run on q_rot
+and K rounded to bf16 by the oracle itself (which isolates the attention
+kernel's error from the rounding of the published format). Small cases cover every round of fill and steady state with
 several key tiles and ragged tails; full-size cases check sampled rows in the
 launch configuration that bench.py times."""
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -18,12 +21,27 @@ pytestmark = pytest.mark.gpu
 
 BF16_ABS, BF16_REL = 2e-2, 1e-2
 F32_ABS = 1e-5
+# With 5% of K rows scaled x8 the softmax is sharply peaked and rounding the
+# rotated q and k to bf16 (the published format) moves each dominant logit by
+# about 8 * 2^-9; near-tied dominant keys then shift outputs of size ~3 by a few
+# 1e-2 against the exact float64 result, whatever the kernel does. So every
+# bf16 case is checked twice: against the oracle run on bf16-rounded q_rot and
+# K (the kernel's own error: max-abs 2e-2, rel-L2 1e-2), and against the exact
+# oracle (rel-L2 1e-2; max-abs 2e-2 on top of the rounding effect
+# |O_exact - O_bf16| that the oracle itself computes).
 
 
-def _compare(ro: Rollout, heads, rows=None, gpu_operands=True):
+def _log(name, **kw):
+    path = os.environ.get("WF_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(dict(test=name, **kw)) + "\n")
+
+
+def _compare(ro: Rollout, heads, rows=None, gpu_operands=True, name=""):
     c = ro.cfg
     want = ro.oracle_out(heads, rows)
-    want_g = ro.oracle_out_from_gpu_operands(heads, rows) if gpu_operands else None
+    want_g = ro.oracle_out_bf16_operands(heads, rows) if gpu_operands else None
     out = tensor_f64(ro.out)
     live = {p.slot for p in ro.layout() if p.slot is not None}
     for s in range(c.num_slots):
@@ -32,15 +50,27 @@ def _compare(ro: Rollout, heads, rows=None, gpu_operands=True):
             assert np.isnan(got_s).all(), f"idle slot {s} was written"
             continue
         assert np.isfinite(got_s).all(), s
-        err = np.abs(got_s - want[s]).max()
+        err = float(np.abs(got_s - want[s]).max())
         if c.dtype == "f32":
+            _log(name, round=ro.round, slot=s, max_abs=err)
             assert err <= F32_ABS, (s, err)
+            continue
+        r = rel_l2(got_s, want[s])
+        rec = dict(round=ro.round, slot=s, max_abs=err, rel_l2=r)
+        if want_g is not None:
+            rec.update(max_abs_bf16_operands=float(np.abs(got_s - want_g[s]).max()),
+                       rel_l2_bf16_operands=rel_l2(got_s, want_g[s]),
+                       rounding_effect=float(np.abs(want_g[s] - want[s]).max()))
+        _log(name, **rec)
+        assert r <= BF16_REL, (s, rec)
+        if want_g is None:
+            assert err <= BF16_ABS, (s, rec)
         else:
-            r = rel_l2(got_s, want[s])
-            assert err <= BF16_ABS and r <= BF16_REL, (s, err, r)
-            if want_g is not None:
-                rg = rel_l2(got_s, want_g[s])
-                assert np.abs(got_s - want_g[s]).max() <= BF16_ABS and rg <= BF16_REL, (s, rg)
+            assert (np.abs(got_s - want[s]) <= BF16_ABS + np.abs(want_g[s] - want[s])).all(), (s, rec)
+            assert rec["max_abs_bf16_operands"] <= BF16_ABS, (s, rec)
+            assert rec["rel_l2_bf16_operands"] <= BF16_REL, (s, rec)
+            if c.k_outlier_frac == 0:
+                assert err <= BF16_ABS, (s, rec)
 
 
 def test_tiny_f32_every_round():
@@ -51,7 +81,7 @@ def test_tiny_f32_every_round():
         ro.attention(0)
         torch.cuda.synchronize()
         assert ro.pool.check_status() == 0
-        _compare(ro, range(cfg.num_heads), gpu_operands=False)
+        _compare(ro, range(cfg.num_heads), gpu_operands=False, name="tiny_f32")
         ro.advance()
     ro.close()
 
@@ -75,7 +105,7 @@ def test_bf16_every_round_small(cfg):
         ro.attention(0)
         torch.cuda.synchronize()
         assert ro.pool.check_status() == 0
-        _compare(ro, range(cfg.num_heads))
+        _compare(ro, range(cfg.num_heads), name="small_bf16")
         ro.advance()
     ro.close()
 
@@ -109,7 +139,7 @@ def test_full_size_sampled(name):
     ro = _steady(cfg)
     heads = sorted({0, cfg.num_heads // 2, cfg.num_heads - 1})
     rows = _sample_rows(cfg.chunk_tokens, 40, 1)
-    _compare(ro, heads, rows)
+    _compare(ro, heads, rows, name=name)
     ro.close()
 
 

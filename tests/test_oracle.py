@@ -311,3 +311,15 @@ def test_publish_pages_layout():
     np.testing.assert_array_equal(pv[3, 0, 1], v[9, 0])
     assert (pk[3, :, 2:] == 0).all() and (pv[3, :, 2:] == 0).all()
     assert np.isnan(pk[1]).all()
+
+
+def test_round_bf16_matches_library_cast():
+    # the library's float32 -> bfloat16 cast rounds to nearest even too
+    x = np.concatenate([_rand(20000, 4) * 10.0 ** np.random.default_rng(5).integers(-3, 4, 20000),
+                        [1.0, -2.5, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 3.0 * 2 ** -9]])
+    x32 = x.astype(np.float32).astype(np.float64)      # exactly representable in fp32
+    ref = torch.from_numpy(x32).float().to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(O.round_bf16(x32), ref)
+    # ties: 1 + 2^-8 is halfway between 1 and 1 + 2^-7 -> even (1.0)
+    assert O.round_bf16(np.array([1.0 + 2 ** -8]))[0] == 1.0
+    assert O.round_bf16(np.array([1.0 + 3 * 2 ** -8]))[0] == 1.0 + 2 ** -6

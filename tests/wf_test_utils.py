@@ -143,19 +143,16 @@ class Rollout:
         q_rot, keys, vals = self.oracle_tensors(heads)
         return O.attention_slot_prefix(q_rot, keys, vals, self.layout(), rows=rows)
 
-    def oracle_out_from_gpu_operands(self, heads: Sequence[int], rows=None):
-        """Oracle attention fed the GPU's own rounded q_rot and K/V pages."""
-        c, hs = self.cfg, list(heads)
-        pages = self.pool.pages_view()
-        qr = tensor_f64(self.q_rot)
-        q_rot, keys, vals = {}, {}, {}
-        for s in self.live:
-            q_rot[s] = qr[s][:, hs]
-        for kind, chunk, slot, tag, pgs in self.pool.layout():
-            kp = tensor_f64(pages[0, pgs, 0][:, hs])   # [npc][heads][P][d]
-            vp = tensor_f64(pages[0, pgs, 1][:, hs])
-            keys[chunk] = np.transpose(kp, (0, 2, 1, 3)).reshape(-1, len(hs), c.head_dim)[:c.chunk_tokens]
-            vals[chunk] = np.transpose(vp, (0, 2, 1, 3)).reshape(-1, len(hs), c.head_dim)[:c.chunk_tokens]
+    def oracle_out_bf16_operands(self, heads: Sequence[int], rows=None):
+        """Oracle attention on operands rounded to the published bf16 format.
+
+        The oracle rotates q and k in float64 and rounds them to bf16 itself
+        (round_bf16), modelling the storage format of q_rot and the K pages;
+        nothing here is read back from the GPU.
+        """
+        q_rot, keys, vals = self.oracle_tensors(heads)
+        q_rot = {s: O.round_bf16(x) for s, x in q_rot.items()}
+        keys = {c: O.round_bf16(x) for c, x in keys.items()}
         return O.attention_slot_prefix(q_rot, keys, vals, self.layout(), rows=rows)
 
     def close(self):
