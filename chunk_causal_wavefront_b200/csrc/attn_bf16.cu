@@ -4,24 +4,31 @@
 // section: full attention inside each chunk, chunk-wise causal attention across
 // chunks with M_WF(s, j) = 1[j >= s]; the ordered context of "Como funciona"
 // (anchor || history || store || denoising K/V) makes the keys of query slot s
-// a prefix of the context, so masked (s, j) chunk pairs are simply never
-// visited: the loop over key tiles stops at the slot's own chunk.
+// a prefix of the context, so masked (s, j) chunk pairs are never visited: the
+// key loop stops at the slot's own chunk.
 //
-// One CTA computes O = softmax(Q K^T / sqrt(d)) V for one 128-row query tile
-// of one (slot, head) with the flash-attention online softmax:
-//   warp 4 (one lane)  TMA producer: Q once, then for every key tile (one
-//                      128-token page) K and V through the page table into a
-//                      two-stage shared-memory ring (128-byte swizzle);
-//   warp 5 (one lane)  tcgen05 issuer: S = Q K^T into one of two TMEM S
-//                      buffers (so S(j+1) overlaps the softmax of tile j), and
-//                      O += P V into a TMEM O accumulator;
-//   warps 0-3          softmax: thread r owns query row r (TMEM lane r); row
-//                      max and sum are thread-local over its 128 columns; P is
-//                      rounded to bf16 and written to shared memory in the
-//                      swizzled K-major layout the tensor core reads; O is
-//                      rescaled in TMEM only when the running max grows by more
-//                      than 2^8 (the exponentials stay <= 256 otherwise); the
-//                      epilogue divides by the row sum and stores bf16 rows.
+// One CTA computes O = softmax(Q K^T / sqrt(d)) V for two 128-row query tiles
+// (q = 0, 1) of one (slot, head), sharing every K/V page it loads:
+//   warp 8 (one lane)  TMA producer: Q0, Q1 once, then for every key tile (one
+//                      128-token page, found through the page table) K and V
+//                      into a two-stage shared-memory ring (128-byte swizzle).
+//   warp 9 (one lane)  tcgen05 issuer, in the order
+//                        S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ...
+//                      S_q = Q_q K^T goes to TMEM columns [128q, 128q+128);
+//                      PV_q reads P_q from TMEM (the first 64 columns of S_q,
+//                      bf16 pairs) and accumulates O_q in columns 256 + 128q.
+//                      While softmax q works on S_q(j+1), the tensor pipe runs
+//                      the other tile's P*V and S (ping-pong).
+//   warps 0-3 / 4-7    softmax of tile 0 / tile 1: thread r owns query row r
+//                      (TMEM lane r); row max and sum are thread-local over its
+//                      128 columns; P is rounded to bf16 and stored back into
+//                      TMEM; O is rescaled in TMEM only when the running max
+//                      grows by more than 2^8 (the exponentials stay <= 256
+//                      otherwise), which is the only time softmax waits for the
+//                      previous P*V. The epilogue divides by the row sum, stages
+//                      the bf16 rows in the tile's (now idle) Q buffer and each
+//                      warp writes its 32 rows with a TMA store that clips rows
+//                      past C.
 // Every wait is bounded: on timeout the CTA records WF_ERR_TIMEOUT, the other
 // roles see the abort flag, in-flight copies and MMAs are drained and TMEM is
 // freed before the CTA exits.
@@ -36,21 +43,26 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBM = 128;              // query rows per CTA
+constexpr int kBM = 128;              // query rows per tile
 constexpr int kBN = 128;              // keys per tile (one page)
 constexpr int kHD = 128;              // head dim
 constexpr uint32_t kHalf = 16384;     // one [128 rows][64 cols] bf16 swizzled block
 constexpr uint32_t kTile = 2 * kHalf; // [128][128] bf16
 constexpr int kPageCache = 1024;      // page ids cached in shared memory
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr long long kWaitLimit = 2000000000LL;  // ~1 s at 2 GHz
 
+// TMEM columns.
+constexpr uint32_t kTmemS = 0;        // S_q at 128 q; P_q aliases its first 64 columns
+constexpr uint32_t kTmemO = 256;      // O_q at 256 + 128 q
+
 // Shared-memory map (offsets from a 1024-byte aligned base).
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTile;          // 2 stages
-constexpr uint32_t kOffV = kOffK + 2 * kTile;      // 2 stages
-constexpr uint32_t kOffP = kOffV + 2 * kTile;
-constexpr uint32_t kOffBar = kOffP + kTile;
+constexpr uint32_t kOffQ = 0;                       // Q0, Q1
+constexpr uint32_t kOffK = kOffQ + 2 * kTile;       // 2 stages
+constexpr uint32_t kOffV = kOffK + 2 * kTile;       // 2 stages
+constexpr uint32_t kOffBar = kOffV + 2 * kTile;
 constexpr int kNumBars = 16;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffPages = kOffMisc + 64;
@@ -58,7 +70,7 @@ constexpr uint32_t kSmemBytes = kOffPages + kPageCache * 4 + 1024;   // + alignm
 
 enum Bar {
   kQFull = 0, kKFull0 = 1, kKEmpty0 = 3, kVFull0 = 5, kVEmpty0 = 7,
-  kSFull0 = 9, kSFree0 = 11, kPFull = 13, kPVDone = 14, kDrain = 15
+  kSFull0 = 9, kPReady0 = 11, kPVDone0 = 13, kDrain = 15
 };
 
 struct Ctx {
@@ -104,6 +116,11 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);   // RNE, lo in the low half
+  return *reinterpret_cast<uint32_t *>(&b);
+}
+
 // Keep the compiler from using tcgen05.ld results before tcgen05.wait::ld.
 #define WF_REG_FENCE8(r, o)                                                                 \
   asm volatile("" : "+r"(r[o + 0]), "+r"(r[o + 1]), "+r"(r[o + 2]), "+r"(r[o + 3]),         \
@@ -118,7 +135,8 @@ __device__ __forceinline__ void reg_fence32(uint32_t *r) {
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bf16_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tq,
-                     const __grid_constant__ CUtensorMap tkv) {
+                     const __grid_constant__ CUtensorMap tkv,
+                     const __grid_constant__ CUtensorMap tout) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -129,19 +147,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // Work item: head-major; inside a head, slots in decreasing context length
-  // (slot 0 first: longest first), then query tiles.
+  // (slot 0 first: longest first), then pairs of query tiles.
   const int tiles = (p.C + kBM - 1) / kBM;
-  const int per_head = p.live.n * tiles;
+  const int pairs = (tiles + 1) / 2;
+  const int per_head = p.live.n * pairs;
   const int h = blockIdx.x / per_head;
   const int rem = blockIdx.x - h * per_head;
-  const int li = p.live.n - 1 - rem / tiles;
-  const int tile = rem % tiles;
+  const int li = p.live.n - 1 - rem / pairs;
+  const int pair = rem % pairs;
   const int slot = p.live.slot[li];
   const int npos = p.live.npos[li];
-  const int row0 = tile * kBM;
+  const int row0 = pair * 2 * kBM;
+  const bool has_q1 = 2 * pair + 1 < tiles;
 
   // Readiness + bounds check of the whole round's context (so that a stale
-  // page stops every CTA of the launch), caching this item's page ids.
+  // page stops every CTA of the launch), caching the page ids.
   {
     int bad = 0, stale = 0;
     const int total = p.n_pos * p.npc;
@@ -155,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
       *abort_flag = 0;
       for (int b = 0; b < kNumBars; ++b) {
-        const bool softmax_arrives = b == kSFree0 || b == kSFree0 + 1 || b == kPFull;
+        const bool softmax_arrives = b == kPReady0 || b == kPReady0 + 1;
         mbar_init(bars + b, softmax_arrives ? kBM : 1);
       }
       fence_barrier_init();
@@ -167,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       return;
     }
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -179,21 +199,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tiles = npos * p.npc;
   const int last_valid = p.C - (p.npc - 1) * p.P;   // keys in a chunk's last page
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tkv);
+      tma_prefetch_desc(&tout);
       uint8_t *sQ = smem + kOffQ;
-      mbar_arrive_expect_tx(bars + kQFull, kTile);
+      mbar_arrive_expect_tx(bars + kQFull, has_q1 ? 2 * kTile : kTile);
       tma_load_4d(sQ, &tq, bars + kQFull, 0, h, row0, slot);
       tma_load_4d(sQ + kHalf, &tq, bars + kQFull, 64, h, row0, slot);
+      if (has_q1) {
+        tma_load_4d(sQ + kTile, &tq, bars + kQFull, 0, h, row0 + kBM, slot);
+        tma_load_4d(sQ + kTile + kHalf, &tq, bars + kQFull, 64, h, row0 + kBM, slot);
+      }
       int nk[2] = {0, 0}, nv[2] = {0, 0};
       for (int j = 0; j < n_tiles; ++j) {
         const int stg = j & 1;
         const uint32_t ph = (j >> 1) & 1;
-        const int idx = j;   // (position, page) flattened == tile index
-        const int phys = idx < kPageCache ? page_cache[idx] : __ldcg(p.table + kTabPages + idx);
+        const int phys = j < kPageCache ? page_cache[j] : __ldcg(p.table + kTabPages + j);
         const int rowk = static_cast<int>(p.layer_row0) + ((phys * 2) * p.Hh + h) * p.P;
         const int rowv = rowk + p.Hh * p.P;
         uint8_t *sK = smem + kOffK + stg * kTile;
@@ -216,165 +240,187 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       drain_wait(ctx, kQFull, 0);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- MMA issuer --
     if (lane == 0) {
       constexpr uint32_t idS = make_idesc_bf16(kBM, kBN, false);
       constexpr uint32_t idPV = make_idesc_bf16(kBM, kHD, true);
-      const uint32_t tO = tmem + 256;
       const uint32_t aQ = smem_u32(smem + kOffQ);
-      const uint32_t aP = smem_u32(smem + kOffP);
-      bool ok = wait_bar(ctx, kQFull, 0);
-      tc_fence_after();
-      auto issue_s = [&](int j) -> bool {
-        const int stg = j & 1, b = j & 1;
-        if (!wait_bar(ctx, kKFull0 + stg, (j >> 1) & 1)) return false;
-        if (j >= 2 && !wait_bar(ctx, kSFree0 + b, ((j - 2) >> 1) & 1)) return false;
-        tc_fence_after();
-        const uint32_t aK = smem_u32(smem + kOffK + stg * kTile);
+      auto issue_s = [&](int q, int j) {
+        const uint32_t aK = smem_u32(smem + kOffK + (j & 1) * kTile);
 #pragma unroll
         for (int k = 0; k < kHD / 16; ++k) {
           const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
-          mma_bf16_ss(tmem + b * 128, make_desc_sw128(aQ + off, 16, 1024),
+          mma_bf16_ss(tmem + kTmemS + q * 128, make_desc_sw128(aQ + q * kTile + off, 16, 1024),
                       make_desc_sw128(aK + off, 16, 1024), idS, k > 0);
         }
-        mma_commit(bars + kSFull0 + b);
-        mma_commit(bars + kKEmpty0 + stg);
-        return true;
+        mma_commit(bars + kSFull0 + q);
       };
-      if (ok && n_tiles > 0) ok = issue_s(0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles && !issue_s(j + 1)) break;
-        const int stg = j & 1;
-        if (!wait_bar(ctx, kPFull, j & 1)) break;
-        if (!wait_bar(ctx, kVFull0 + stg, (j >> 1) & 1)) break;
-        tc_fence_after();
-        const uint32_t aV = smem_u32(smem + kOffV + stg * kTile);
+      auto issue_pv = [&](int q, int j) {
+        const uint32_t aV = smem_u32(smem + kOffV + (j & 1) * kTile);
 #pragma unroll
         for (int k = 0; k < kBN / 16; ++k) {
-          const uint64_t da = make_desc_sw128(aP + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
-          const uint64_t db = make_desc_sw128(aV + k * 2048, kHalf, 1024);
-          mma_bf16_ss(tO, da, db, idPV, (j > 0 || k > 0) ? 1u : 0u);
+          // A = P_q from TMEM: 16 keys = 8 columns of bf16 pairs per step.
+          mma_bf16_ts(tmem + kTmemO + q * 128, tmem + kTmemS + q * 128 + k * 8,
+                      make_desc_sw128(aV + k * 2048, kHalf, 1024), idPV,
+                      (j > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(bars + kPVDone0 + q);
+      };
+      bool ok = wait_bar(ctx, kQFull, 0) && wait_bar(ctx, kKFull0, 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (has_q1) issue_s(1, 0);
+        mma_commit(bars + kKEmpty0);
+      }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int stg = j & 1;
+        const bool more = j + 1 < n_tiles;
+        if (!wait_bar(ctx, kVFull0 + stg, (j >> 1) & 1)) break;
+        if (!wait_bar(ctx, kPReady0, j & 1)) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (more) {
+          if (!wait_bar(ctx, kKFull0 + ((j + 1) & 1), ((j + 1) >> 1) & 1)) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (has_q1) {
+          if (!wait_bar(ctx, kPReady0 + 1, j & 1)) break;
+          tc_fence_after();
+          issue_pv(1, j);
+          if (more) issue_s(1, j + 1);
         }
         mma_commit(bars + kVEmpty0 + stg);
-        mma_commit(bars + kPVDone);
+        if (more) mma_commit(bars + kKEmpty0 + ((j + 1) & 1));
       }
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
       mma_commit(bars + kDrain);
       drain_wait(ctx, kDrain, 0);
     }
-  } else {
+  } else if (warp < 4 || has_q1) {
     // ------------------------------------------------------------- softmax --
-    const int r = warp * 32 + lane;                     // query row == TMEM lane
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-    uint8_t *sP = smem + kOffP;
+    const int q = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;               // query row == TMEM lane
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + kTmemS + q * 128;
+    const uint32_t tO = tmem + lane_addr + kTmemO + q * 128;
     float m = -INFINITY, l = 0.0f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      const int b = j & 1;
-      ok = __all_sync(0xffffffffu, wait_bar(ctx, kSFull0 + b, (j >> 1) & 1));
+      ok = __all_sync(0xffffffffu, wait_bar(ctx, kSFull0 + q, j & 1));
       if (!ok) break;
       tc_fence_after();
       uint32_t s[128];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_addr + b * 128 + c * 32, s + c * 32);
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s + c * 32);
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence32(s + c * 32);
-      tc_fence_before();
-      mbar_arrive(bars + kSFree0 + b);
 
       const int valid = (j % p.npc == p.npc - 1) ? last_valid : kBN;
+      if (valid < kBN) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) s[c] = __float_as_uint(-INFINITY);
+      }
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        if (c >= valid) s[c] = __float_as_uint(-INFINITY);
-        mx = fmaxf(mx, __uint_as_float(s[c]));
-      }
+      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
       const float m_new = fmaxf(m, mx * p.scale_log2);
-      const bool rescale = (j == 0) || (m_new - m > 8.0f);
+      const bool rescale = m_new - m > 8.0f;             // always true on the first tile
       const float alpha = rescale ? ex2(m - m_new) : 1.0f;
       const float m_use = rescale ? m_new : m;
-      float rowsum = 0.0f;
-      uint32_t pw[64];
+      float sum0 = 0.0f, sum1 = 0.0f;
+      // P = 2^(s * log2(e) / sqrt(d) - m), rounded to bf16 pairs and streamed
+      // back into the first 64 columns of S_q, 16 columns (32 keys) at a time.
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2(fmaf(__uint_as_float(s[2 * c]), p.scale_log2, -m_use));
-        const float p1 = ex2(fmaf(__uint_as_float(s[2 * c + 1]), p.scale_log2, -m_use));
-        __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-        pw[c] = *reinterpret_cast<uint32_t *>(&pb);
-        rowsum += __uint_as_float(pw[c] << 16) + __uint_as_float(pw[c] & 0xFFFF0000u);
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t pw[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int k0 = cc * 32 + 2 * c;
+          const float p0 = ex2(fmaf(__uint_as_float(s[k0]), p.scale_log2, -m_use));
+          const float p1 = ex2(fmaf(__uint_as_float(s[k0 + 1]), p.scale_log2, -m_use));
+          sum0 += p0;
+          sum1 += p1;
+          pw[c] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tS + cc * 16, pw);
       }
-      l = l * alpha + rowsum;
+      l = l * alpha + (sum0 + sum1);
       m = m_use;
 
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, wait_bar(ctx, kPVDone, (j - 1) & 1));
+      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+        // O_q must hold P*V up to tile j-1 before it is rescaled.
+        ok = __all_sync(0xffffffffu, wait_bar(ctx, kPVDone0 + q, (j - 1) & 1));
         if (!ok) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_addr + 256 + c * 32, o);
-            tmem_ld_wait();
-            reg_fence32(o);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_ld_wait();
+          reg_fence32(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tmem + lane_addr + 256 + c * 32, o);
-          }
-          tmem_st_wait();
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + c * 32, o);
         }
       }
-      // P row -> shared memory, K-major with the 128-byte swizzle: 16-byte
-      // chunk c of row r in 64-key half kt lands at r*128 + ((c ^ (r & 7)) * 16).
-#pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        const int kt = cc >> 3, c = cc & 7;
-        const uint32_t addr = smem_u32(sP + kt * kHalf + r * 128 + ((c ^ (r & 7)) << 4));
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pw[4 * cc]),
-                     "r"(pw[4 * cc + 1]), "r"(pw[4 * cc + 2]), "r"(pw[4 * cc + 3])
-                     : "memory");
-      }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bars + kPFull);
+      mbar_arrive(bars + kPReady0 + q);
     }
     if (ok && n_tiles > 0) {
-      ok = __all_sync(0xffffffffu, wait_bar(ctx, kPVDone, (n_tiles - 1) & 1));
+      ok = __all_sync(0xffffffffu, wait_bar(ctx, kPVDone0 + q, (n_tiles - 1) & 1));
     }
     if (ok && n_tiles > 0) {
       tc_fence_after();
       const float inv = 1.0f / l;
-      const int n = row0 + r;
-      __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) +
-                           ((static_cast<size_t>(slot) * p.C + n) * p.Hh + h) * kHD;
+      // Stage the bf16 rows in this tile's Q buffer (its last reader, the final
+      // S MMA, has completed) in the 128-byte swizzled layout of the output
+      // tensor map, whose box is 32 rows: 16-byte chunk c of row r in 64-column
+      // half kt lands at kt * 16 KB + r * 128 + ((c ^ (r & 7)) * 16), so each
+      // warp's 32 rows form one contiguous 4 KB box per half and the warp
+      // stores them itself (no cross-warp barrier).
+      uint8_t *stage = smem + kOffQ + q * kTile;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_addr + 256 + c * 32, o);
+        tmem_ld32(tO + c4 * 32, o);
         tmem_ld_wait();
         reg_fence32(o);
         uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv,
-                                                   __uint_as_float(o[2 * i + 1]) * inv);
-          w[i] = *reinterpret_cast<uint32_t *>(&v);
-        }
-        if (n < p.C) {
-          uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 32);
+        for (int i = 0; i < 16; ++i)
+          w[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        for (int i = 0; i < 4; ++i) {
+          const int cc = c4 * 4 + i;                      // 16-byte chunk 0..15 of the row
+          const int kt = cc >> 3, c = cc & 7;
+          const uint32_t addr = smem_u32(stage + kt * kHalf + r * 128 + ((c ^ (r & 7)) << 4));
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[4 * i]),
+                       "r"(w[4 * i + 1]), "r"(w[4 * i + 2]), "r"(w[4 * i + 3])
+                       : "memory");
         }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      const int wr = (warp & 3) * 32;                     // this warp's first row in the tile
+      if (lane == 0 && row0 + q * kBM + wr < p.C) {       // boxes wholly past C are skipped
+        tma_store_4d(&tout, stage + wr * 128, 0, h, row0 + q * kBM + wr, slot);
+        tma_store_4d(&tout, stage + kHalf + wr * 128, 64, h, row0 + q * kBM + wr, slot);
+        tma_store_commit();
+        tma_store_wait_all();
+      }
+      __syncwarp();
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -383,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_attention_bf16(const AttnParams &p, const void *tmap_q, const void *tmap_kv,
-                                  cudaStream_t st) {
+                                  const void *tmap_out, cudaStream_t st) {
   if (p.live.n == 0) return cudaSuccess;
   if (p.d != kHD || p.P != kBN) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel,
@@ -391,10 +437,11 @@ cudaError_t launch_attention_bf16(const AttnParams &p, const void *tmap_q, const
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   const int tiles = (p.C + kBM - 1) / kBM;
-  const int64_t blocks = static_cast<int64_t>(tiles) * p.live.n * p.Hh;
+  const int64_t blocks = static_cast<int64_t>((tiles + 1) / 2) * p.live.n * p.Hh;
   if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
   attn_bf16_kernel<<<static_cast<unsigned>(blocks), kThreads, kSmemBytes, st>>>(
-      p, *static_cast<const CUtensorMap *>(tmap_q), *static_cast<const CUtensorMap *>(tmap_kv));
+      p, *static_cast<const CUtensorMap *>(tmap_q), *static_cast<const CUtensorMap *>(tmap_kv),
+      *static_cast<const CUtensorMap *>(tmap_out));
   return cudaGetLastError();
 }
 

@@ -438,7 +438,10 @@ wf_status wf_round_attention(wf_pool *p, int32_t layer, const void *q_rot, void 
     const cuuint32_t box[4] = {64, 1, 128, 1};
     if (!encode_bf16_map(&qmap, const_cast<void *>(q_rot), 4, dims, strides, box))
       return WF_ERR_CUDA;
-    e = launch_attention_bf16(ap, &qmap, &p->kv_map, cs);
+    CUtensorMap omap;
+    const cuuint32_t obox[4] = {64, 1, 32, 1};
+    if (!encode_bf16_map(&omap, out, 4, dims, strides, obox)) return WF_ERR_CUDA;
+    e = launch_attention_bf16(ap, &qmap, &p->kv_map, &omap, cs);
   } else {
     e = launch_attention_f32(ap, cs);
   }

@@ -70,9 +70,11 @@ cudaError_t launch_publish_bf16(const PublishParams &p, cudaStream_t st);
 cudaError_t launch_publish_f32(const PublishParams &p, cudaStream_t st);
 cudaError_t launch_attention_f32(const AttnParams &p, cudaStream_t st);
 // The bf16 tensor-core path takes the encoded tensor maps (opaque 128-byte
-// CUtensorMap objects) of q_rot, out and the pool's K/V pages.
+// CUtensorMap objects) of q_rot (box 64 x 1 x 128 rows), the pool's K/V pages
+// (box 64 x 128) and out (box 64 x 1 x 32 rows).
 cudaError_t launch_attention_bf16(const AttnParams &p, const void *tmap_q,
-                                  const void *tmap_kv, cudaStream_t st);
+                                  const void *tmap_kv, const void *tmap_out,
+                                  cudaStream_t st);
 cudaError_t launch_table_upload(int32_t *dst, const int32_t *src, int n_words,
                                 cudaStream_t st);
 cudaError_t launch_poke(int32_t *dst, int32_t value, cudaStream_t st);
