@@ -1,6 +1,7 @@
 """Build libwf.so in-tree with nvcc for sm_100a.
 
-Usage: python -m chunk_causal_wavefront_b200.build [--force] [--verbose]
+Usage: python chunk_causal_wavefront_b200/build.py [--force] [--verbose] [--ptxas-info]
+(run by path, so that a stale libwf.so is not loaded through the package)
 """
 from __future__ import annotations
 

@@ -35,6 +35,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "exp2_poly.cuh"
 #include "sm100.cuh"
 #include "wf_internal.h"
 
@@ -49,9 +50,17 @@ constexpr int kHD = 128;              // head dim
 constexpr uint32_t kHalf = 16384;     // one [128 rows][64 cols] bf16 swizzled block
 constexpr uint32_t kTile = 2 * kHalf; // [128][128] bf16
 constexpr int kPageCache = 1024;      // page ids cached in shared memory
-constexpr int kThreads = 320;
+// Warpgroups 0 and 1 run the softmax of tiles 0 and 1; warpgroup 2 holds the
+// TMA producer (warp 8) and the MMA issuer (warp 9); warps 10-11 only hand
+// their registers over. Launched at 168 registers per thread (384 x 168 =
+// 64512), warpgroup 2 drops to 64 and the softmax warpgroups rise to 216:
+// 256 x 216 + 128 x 64 = 63488.
+constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr uint32_t kRegsSoftmax = 216;
+constexpr uint32_t kRegsControl = 64;
+static_assert(256 * kRegsSoftmax + 128 * kRegsControl <= 384 * 168, "register split");
 constexpr long long kWaitLimit = 2000000000LL;  // ~1 s at 2 GHz
 
 // TMEM columns.
@@ -114,6 +123,12 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -199,7 +214,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tiles = npos * p.npc;
   const int last_valid = p.C - (p.npc - 1) * p.P;   // keys in a chunk's last page
 
-  if (warp == kProducerWarp) {
+  if (warp >= 8) {
+   setmaxnreg_dec<kRegsControl>();
+   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       tma_prefetch_desc(&tq);
@@ -299,7 +316,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bars + kDrain);
       drain_wait(ctx, kDrain, 0);
     }
-  } else if (warp < 4 || has_q1) {
+   }
+  } else {
+   setmaxnreg_inc<kRegsSoftmax>();
+   if (warp < 4 || has_q1) {
     // ------------------------------------------------------------- softmax --
     const int q = warp >> 2;
     const int r = (warp & 3) * 32 + lane;               // query row == TMEM lane
@@ -325,30 +345,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 128; ++c)
           if (c >= valid) s[c] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
+      // Row max: eight independent chains of three-input max, then a tree.
+      float m8[8];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+      for (int i = 0; i < 8; ++i) {
+        float a = max3(__uint_as_float(s[i]), __uint_as_float(s[i + 8]), __uint_as_float(s[i + 16]));
+#pragma unroll
+        for (int b = 24; b < 120; b += 16)
+          a = max3(a, __uint_as_float(s[b + i]), __uint_as_float(s[b + 8 + i]));
+        m8[i] = fmaxf(a, __uint_as_float(s[120 + i]));
+      }
+      const float mx = fmaxf(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], max3(m8[5], m8[6], m8[7])));
       const float m_new = fmaxf(m, mx * p.scale_log2);
       const bool rescale = m_new - m > 8.0f;             // always true on the first tile
       const float alpha = rescale ? ex2(m - m_new) : 1.0f;
       const float m_use = rescale ? m_new : m;
-      float sum0 = 0.0f, sum1 = 0.0f;
-      // P = 2^(s * log2(e) / sqrt(d) - m), rounded to bf16 pairs and streamed
+      // P = 2^(s * log2(e) / sqrt(d) - m), in packed pairs: 3 of every 4 pairs
+      // on the MUFU unit, 1 on the FMA pipe; rounded to bf16 pairs and streamed
       // back into the first 64 columns of S_q, 16 columns (32 keys) at a time.
+      const uint64_t sc2 = f2(p.scale_log2, p.scale_log2), nm2 = f2(-m_use, -m_use);
+      uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t pw[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const int k0 = cc * 32 + 2 * c;
-          const float p0 = ex2(fmaf(__uint_as_float(s[k0]), p.scale_log2, -m_use));
-          const float p1 = ex2(fmaf(__uint_as_float(s[k0 + 1]), p.scale_log2, -m_use));
-          sum0 += p0;
-          sum1 += p1;
-          pw[c] = pack_bf16(p0, p1);
+          const uint64_t x2 = ffma2(f2(__uint_as_float(s[k0]), __uint_as_float(s[k0 + 1])), sc2, nm2);
+          uint64_t e2;
+          if ((c & 3) == 3) {
+            e2 = ex2_poly2(x2);
+          } else {
+            float a, b;
+            unf2(x2, a, b);
+            e2 = f2(ex2(a), ex2(b));
+          }
+          acc[c & 3] = fadd2(acc[c & 3], e2);
+          float a, b;
+          unf2(e2, a, b);
+          pw[c] = pack_bf16(a, b);
         }
         tmem_st16(tS + cc * 16, pw);
       }
+      float sum0, sum1;
+      unf2(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), sum0, sum1);
       l = l * alpha + (sum0 + sum1);
       m = m_use;
 
@@ -363,8 +403,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tO + c * 32, o);
           tmem_ld_wait();
           reg_fence32(o);
+          const uint64_t a2 = f2(alpha, alpha);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          for (int i = 0; i < 32; i += 2) {
+            const uint64_t v = fmul2(f2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
+            float lo, hi;
+            unf2(v, lo, hi);
+            o[i] = __float_as_uint(lo);
+            o[i + 1] = __float_as_uint(hi);
+          }
           tmem_st32(tO + c * 32, o);
         }
       }
@@ -416,6 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
+   }
   }
 
   tc_fence_before();

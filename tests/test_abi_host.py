@@ -21,7 +21,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def header_functions():
     src = open(os.path.join(ROOT, "include", "wf.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(wf_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(wf_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_library_exports_every_declared_function():
