@@ -35,7 +35,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
-#include "exp2_poly.cuh"
+#include "f32x2.cuh"
 #include "sm100.cuh"
 #include "wf_internal.h"
 
@@ -360,9 +360,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool rescale = m_new - m > 8.0f;             // always true on the first tile
       const float alpha = rescale ? ex2(m - m_new) : 1.0f;
       const float m_use = rescale ? m_new : m;
-      // P = 2^(s * log2(e) / sqrt(d) - m), in packed pairs: 3 of every 4 pairs
-      // on the MUFU unit, 1 on the FMA pipe; rounded to bf16 pairs and streamed
-      // back into the first 64 columns of S_q, 16 columns (32 keys) at a time.
+      // P = 2^(s * log2(e) / sqrt(d) - m) on the MUFU unit, the scale-subtract
+      // and the row sums in packed f32x2 arithmetic; rounded to bf16 pairs and
+      // streamed back into the first 64 columns of S_q, 16 columns (32 keys) at
+      // a time.
       const uint64_t sc2 = f2(p.scale_log2, p.scale_log2), nm2 = f2(-m_use, -m_use);
       uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -372,18 +373,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 16; ++c) {
           const int k0 = cc * 32 + 2 * c;
           const uint64_t x2 = ffma2(f2(__uint_as_float(s[k0]), __uint_as_float(s[k0 + 1])), sc2, nm2);
-          uint64_t e2;
-          if ((c & 3) == 3) {
-            e2 = ex2_poly2(x2);
-          } else {
-            float a, b;
-            unf2(x2, a, b);
-            e2 = f2(ex2(a), ex2(b));
-          }
-          acc[c & 3] = fadd2(acc[c & 3], e2);
           float a, b;
-          unf2(e2, a, b);
-          pw[c] = pack_bf16(a, b);
+          unf2(x2, a, b);
+          const float e0 = ex2(a), e1 = ex2(b);
+          acc[c & 3] = fadd2(acc[c & 3], f2(e0, e1));
+          pw[c] = pack_bf16(e0, e1);
         }
         tmem_st16(tS + cc * 16, pw);
       }

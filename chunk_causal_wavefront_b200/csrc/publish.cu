@@ -6,9 +6,10 @@
 // by a ready signal. Here the "slots" are the pages that the device page table
 // assigns to each live slot; the ready signal is a per-page tag.
 //
-// One launch covers every live slot of the round. Each thread owns one
-// 16-byte vector (8 bf16 or 4 fp32 values = 4 or 2 rotary pairs) of one
-// (slot, token, head) row: it loads q, k and v with streaming 16-byte loads,
+// One launch covers every live slot of the round (grid row = slot). A thread
+// handles 16-byte vectors (8 bf16 or 4 fp32 values = 4 or 2 rotary pairs) of
+// (slot, token, head) rows, two per iteration: it loads q, k and v with
+// streaming 16-byte loads,
 // rotates q and k in fp32 with (cos, sin) tables computed on the host in fp64,
 // rounds once to the storage type and issues 16-byte stores to q_rot and to
 // the K and V pages. Consecutive threads cover consecutive 16-byte vectors of
@@ -78,75 +79,110 @@ __device__ __forceinline__ void rope_vec(float *x, int dim0, int tpos, int ypos,
   }
 }
 
+// Physical page holding page j of live slot li's chunk (-1 if the table is bad).
+__device__ __forceinline__ int slot_page(const PublishParams &p, int pos, int j) {
+  const int phys = pos < 0 ? -1 : __ldg(p.table + kTabPages + pos * p.npc + j);
+  return (phys < 0 || phys >= p.num_pages) ? -1 : phys;
+}
+
+// One main-part vector: rotate q and k, write q_rot and the K/V page rows.
+template <typename T>
+__device__ __forceinline__ void publish_vector(const PublishParams &p, int li, int pos, int n,
+                                               int h, int e, const uint4 &qv, const uint4 &kv,
+                                               const uint4 &vv, size_t src) {
+  constexpr int N = Vec<T>::N;
+  float q[N], k[N];
+  unpack(qv, q, T());
+  unpack(kv, k, T());
+  if (p.rope) {
+    const int hw = p.gh * p.gw;
+    const int tpos = p.F * p.live.chunk[li] + n / hw;
+    const int ypos = (n / p.gw) % p.gh;
+    const int xpos = n % p.gw;
+    rope_vec<N>(q, e * N, tpos, ypos, xpos, p);
+    rope_vec<N>(k, e * N, tpos, ypos, xpos, p);
+  }
+  *reinterpret_cast<uint4 *>(static_cast<T *>(p.q_rot) + src) = pack(q, T());
+  const int j = n / p.P, row = n - j * p.P;
+  const int phys = slot_page(p, pos, j);
+  if (phys < 0) {
+    record_status(p.status, WF_ERR_BAD_PAGE);
+    return;
+  }
+  const size_t page_elems = static_cast<size_t>(2) * p.Hh * p.P * p.d;
+  T *kdst = reinterpret_cast<T *>(p.pages) + phys * page_elems +
+            (static_cast<size_t>(h) * p.P + row) * p.d + e * N;
+  T *vdst = kdst + static_cast<size_t>(p.Hh) * p.P * p.d;
+  *reinterpret_cast<uint4 *>(kdst) = pack(k, T());
+  *reinterpret_cast<uint4 *>(vdst) = vv;
+  if (row == 0 && h == 0 && e == 0) p.tags[phys] = p.live.tag[li];
+}
+
+// Grid: (blocks, live slots). Each thread walks its slot's vectors with a
+// grid stride, two at a time so that six 16-byte loads are in flight before
+// the first one is used. Vector v < C * heads * d/N is (token n, head h,
+// vector e) of the [C][heads][d] rows; the remaining vectors zero the rows
+// past C in the chunk's last page (K then V, head-major, row, vector).
 template <typename T>
 __global__ void __launch_bounds__(256) publish_kernel(const PublishParams p) {
   constexpr int N = Vec<T>::N;
+  const int li = blockIdx.y;
+  const int slot = p.live.slot[li];
+  const int pos = __ldg(p.table + kTabSlotPos + slot);
   const int vpr = p.d / N;                                   // vectors per head row
-  const int64_t per_slot = static_cast<int64_t>(p.C) * p.Hh * vpr;
-  const int64_t main_n = per_slot * p.live.n;
-  const int tail_rows = p.npc * p.P - p.C;                   // zero rows of the last page
-  const int64_t tail_per_slot = static_cast<int64_t>(2) * p.Hh * tail_rows * vpr;
-  const int64_t total = main_n + tail_per_slot * p.live.n;
-  const size_t page_elems = static_cast<size_t>(2) * p.Hh * p.P * p.d;
-  T *pages = reinterpret_cast<T *>(p.pages);
+  const int vpt = p.Hh * vpr;                                // vectors per token
+  const int main_n = p.C * vpt;
+  const int tail_rows = p.npc * p.P - p.C;
+  const int total = main_n + 2 * p.Hh * tail_rows * vpr;
+  const size_t slot_off = static_cast<size_t>(slot) * p.C * p.Hh * p.d;
+  const T *qs = static_cast<const T *>(p.q) + slot_off;
+  const T *ks = static_cast<const T *>(p.k) + slot_off;
+  const T *vs = static_cast<const T *>(p.v) + slot_off;
+  const int stride = gridDim.x * blockDim.x;
 
-  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    if (idx < main_n) {
-      const int li = static_cast<int>(idx / per_slot);
-      int64_t r = idx - li * per_slot;
-      const int e = static_cast<int>(r % vpr);
-      r /= vpr;
-      const int h = static_cast<int>(r % p.Hh);
-      const int n = static_cast<int>(r / p.Hh);
-      const int slot = p.live.slot[li];
-      const int pos = __ldg(p.table + kTabSlotPos + slot);
-      const int j = n / p.P, row = n - j * p.P;
-      const int phys = pos < 0 ? -1 : __ldg(p.table + kTabPages + pos * p.npc + j);
-      const size_t src = ((static_cast<size_t>(slot) * p.C + n) * p.Hh + h) * p.d + e * N;
-      float q[N], k[N];
-      unpack(ld_stream(static_cast<const T *>(p.q) + src), q, T());
-      unpack(ld_stream(static_cast<const T *>(p.k) + src), k, T());
-      const uint4 v = ld_stream(static_cast<const T *>(p.v) + src);
-      if (p.rope) {
-        const int chunk = p.live.chunk[li];
-        const int hw = p.gh * p.gw;
-        const int tpos = p.F * chunk + n / hw;
-        const int ypos = (n / p.gw) % p.gh;
-        const int xpos = n % p.gw;
-        rope_vec<N>(q, e * N, tpos, ypos, xpos, p);
-        rope_vec<N>(k, e * N, tpos, ypos, xpos, p);
+  for (int v0 = blockIdx.x * blockDim.x + threadIdx.x; v0 < total; v0 += 2 * stride) {
+    const int v1 = v0 + stride;
+    const bool m0 = v0 < main_n, m1 = v1 < main_n;
+    uint4 q0, k0, w0, q1, k1, w1;
+    if (m0) {
+      q0 = ld_stream(qs + static_cast<size_t>(v0) * N);
+      k0 = ld_stream(ks + static_cast<size_t>(v0) * N);
+      w0 = ld_stream(vs + static_cast<size_t>(v0) * N);
+    }
+    if (m1) {
+      q1 = ld_stream(qs + static_cast<size_t>(v1) * N);
+      k1 = ld_stream(ks + static_cast<size_t>(v1) * N);
+      w1 = ld_stream(vs + static_cast<size_t>(v1) * N);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int v = u ? v1 : v0;
+      if (v >= total) break;
+      if (u ? m1 : m0) {
+        const int n = v / vpt;
+        const int rem = v - n * vpt;
+        const int h = rem / vpr;
+        const int e = rem - h * vpr;
+        publish_vector<T>(p, li, pos, n, h, e, u ? q1 : q0, u ? k1 : k0, u ? w1 : w0,
+                          slot_off + static_cast<size_t>(v) * N);
+      } else {
+        int r = v - main_n;
+        const int e = r % vpr;
+        r /= vpr;
+        const int row = p.P - tail_rows + r % tail_rows;
+        r /= tail_rows;
+        const int h = r % p.Hh;
+        const int kv = r / p.Hh;
+        const int phys = slot_page(p, pos, p.npc - 1);
+        if (phys < 0) {
+          record_status(p.status, WF_ERR_BAD_PAGE);
+          continue;
+        }
+        T *dst = reinterpret_cast<T *>(p.pages) +
+                 phys * (static_cast<size_t>(2) * p.Hh * p.P * p.d) +
+                 ((static_cast<size_t>(kv) * p.Hh + h) * p.P + row) * p.d + e * N;
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
       }
-      *reinterpret_cast<uint4 *>(static_cast<T *>(p.q_rot) + src) = pack(q, T());
-      if (phys < 0 || phys >= p.num_pages) {
-        record_status(p.status, WF_ERR_BAD_PAGE);
-        continue;
-      }
-      T *kdst = pages + phys * page_elems + (static_cast<size_t>(h) * p.P + row) * p.d + e * N;
-      T *vdst = kdst + static_cast<size_t>(p.Hh) * p.P * p.d;
-      *reinterpret_cast<uint4 *>(kdst) = pack(k, T());
-      *reinterpret_cast<uint4 *>(vdst) = v;
-      if (row == 0 && h == 0 && e == 0) p.tags[phys] = p.live.tag[li];
-    } else {
-      int64_t r = idx - main_n;
-      const int li = static_cast<int>(r / tail_per_slot);
-      r -= li * tail_per_slot;
-      const int e = static_cast<int>(r % vpr);
-      r /= vpr;
-      const int row = p.P - tail_rows + static_cast<int>(r % tail_rows);
-      r /= tail_rows;
-      const int h = static_cast<int>(r % p.Hh);
-      const int kv = static_cast<int>(r / p.Hh);
-      const int slot = p.live.slot[li];
-      const int pos = __ldg(p.table + kTabSlotPos + slot);
-      const int phys = pos < 0 ? -1 : __ldg(p.table + kTabPages + pos * p.npc + (p.npc - 1));
-      if (phys < 0 || phys >= p.num_pages) {
-        record_status(p.status, WF_ERR_BAD_PAGE);
-        continue;
-      }
-      T *dst = pages + phys * page_elems +
-               ((static_cast<size_t>(kv) * p.Hh + h) * p.P + row) * p.d + e * N;
-      *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
     }
   }
 }
@@ -156,17 +192,20 @@ cudaError_t launch(const PublishParams &p, cudaStream_t st) {
   if (p.live.n == 0) return cudaSuccess;
   constexpr int N = Vec<T>::N;
   const int64_t vpr = p.d / N;
-  const int64_t total = static_cast<int64_t>(p.live.n) *
-                        (static_cast<int64_t>(p.C) * p.Hh * vpr +
-                         2LL * p.Hh * (p.npc * p.P - p.C) * vpr);
-  int sms = 148;
-  int dev;
+  const int64_t per_slot = static_cast<int64_t>(p.C) * p.Hh * vpr +
+                           2LL * p.Hh * (p.npc * p.P - p.C) * vpr;
+  if (per_slot >= (int64_t(1) << 30)) return cudaErrorInvalidValue;   // int32 vector indices
+  int sms = 148, dev = 0, per_sm = 4;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t blocks = (total + 255) / 256;
-  const int64_t cap = static_cast<int64_t>(sms) * 8;   // 8 resident 256-thread blocks per SM
-  if (blocks > cap) blocks = cap;
-  publish_kernel<T><<<static_cast<int>(blocks), 256, 0, st>>>(p);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, publish_kernel<T>, 256, 0);
+  if (per_sm < 1) per_sm = 1;
+  // One wave: every resident block slot of the GPU, spread over the live slots.
+  int64_t bx = (static_cast<int64_t>(sms) * per_sm) / p.live.n;
+  const int64_t need = (per_slot + 511) / 512;            // two vectors per thread
+  if (bx > need) bx = need;
+  if (bx < 1) bx = 1;
+  publish_kernel<T><<<dim3(static_cast<unsigned>(bx), static_cast<unsigned>(p.live.n)), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -52,14 +52,22 @@ class KVPool:
     """A paged K/V pool on one GPU (or host-only bookkeeping when device=None)."""
 
     def __init__(self, cfg: WfPoolConfig, device: Optional[torch.device] = None,
-                 page_order: Optional[Sequence[int]] = None, stream=None):
+                 page_order: Optional[Sequence[int]] = None, stream=None,
+                 mem: Optional[torch.Tensor] = None):
+        """``mem`` reuses an existing uint8 device buffer of at least
+        wf_kv_pool_bytes(cfg) bytes (the pool restarts at round 0 in it)."""
         self.cfg = cfg
         self.nbytes = _wf.wf_kv_pool_bytes(cfg)
         self.device = None if device is None else torch.device(device)
         self.dtype = torch.bfloat16 if cfg.dtype == _wf.WF_DTYPE_BF16 else torch.float32
         self.mem = None
         if self.device is not None:
-            self.mem = torch.empty(self.nbytes, dtype=torch.uint8, device=self.device)
+            if mem is not None:
+                if mem.dtype != torch.uint8 or mem.numel() < self.nbytes or not mem.is_cuda:
+                    raise ValueError("mem must be a CUDA uint8 tensor of at least wf_kv_pool_bytes")
+                self.mem = mem
+            else:
+                self.mem = torch.empty(self.nbytes, dtype=torch.uint8, device=self.device)
             with torch.cuda.device(self.device):
                 self.handle = _wf.wf_kv_pool_create(cfg, self.mem.data_ptr(), self.nbytes,
                                                     page_order, _stream(self.device, stream))

@@ -32,7 +32,6 @@ EXPORTS = (
     "wf_kv_pool_bytes", "wf_kv_pool_create", "wf_publish_kv", "wf_round_attention",
     "wf_advance_round", "wf_pool_check_status", "wf_pool_destroy", "wf_status_string",
     "wf_pool_round", "wf_pool_get_geometry", "wf_pool_get_layout", "wf_pool_debug_poke_page",
-    "wf_debug_exp2_poly",
 )
 
 
@@ -88,7 +87,6 @@ def _load():
         "wf_pool_get_geometry": (I32, [P, ctypes.POINTER(WfPoolGeometry)]),
         "wf_pool_get_layout": (I32, [P, i32p, i32p, i32p, i32p, i32p, i32p, I32]),
         "wf_pool_debug_poke_page": (I32, [P, I32, I32, I32, P]),
-        "wf_debug_exp2_poly": (I32, [P, P, I64, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -185,6 +183,3 @@ def wf_pool_debug_poke_page(pool: int, position: int, j: int, physical: int, str
     return _lib.wf_pool_debug_poke_page(pool, position, j, physical,
                                         ctypes.c_void_p(stream or None))
 
-
-def wf_debug_exp2_poly(x: int, y: int, n: int, stream: int) -> int:
-    return _lib.wf_debug_exp2_poly(x, y, n, ctypes.c_void_p(stream or None))

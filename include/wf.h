@@ -184,13 +184,6 @@ wf_status wf_pool_get_layout(const wf_pool *pool, int32_t *n_positions, int32_t 
 wf_status wf_pool_debug_poke_page(wf_pool *pool, int32_t position, int32_t j,
                                   int32_t physical, wf_stream_t stream);
 
-/* Diagnostic: y[i] = 2^x[i] computed by the polynomial the attention kernel
- * uses for a quarter of its exponentials (range reduction to [-1/2, 1/2] plus a
- * degree-3 minimax polynomial; relative error <= 7.5e-5 for x in [-126, 64];
- * 0 for x < -126). x and y are device arrays of n floats. Not part of the
- * round; no passage of the paper corresponds to it. */
-wf_status wf_debug_exp2_poly(const float *x, float *y, int64_t n, wf_stream_t stream);
-
 #ifdef __cplusplus
 }
 #endif

@@ -38,10 +38,10 @@ def _log(name, **kw):
             f.write(json.dumps(dict(test=name, **kw)) + "\n")
 
 
-def _compare(ro: Rollout, heads, rows=None, gpu_operands=True, name=""):
+def _compare(ro: Rollout, heads, rows=None, gpu_operands=True, name="", layer=0):
     c = ro.cfg
-    want = ro.oracle_out(heads, rows)
-    want_g = ro.oracle_out_bf16_operands(heads, rows) if gpu_operands else None
+    want = ro.oracle_out(heads, rows, layer)
+    want_g = ro.oracle_out_bf16_operands(heads, rows, layer) if gpu_operands else None
     out = tensor_f64(ro.out)
     live = {p.slot for p in ro.layout() if p.slot is not None}
     for s in range(c.num_slots):

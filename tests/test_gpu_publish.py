@@ -33,7 +33,7 @@ def _check_round(ro: Rollout, layer: int = 0, full_rope_check: bool = True):
     for p, pgs, tag in model.table():
         if p.slot is None:
             continue
-        q, k, v, chunk = ro.live[p.slot]
+        q, k, v, chunk = ro.live[layer][p.slot]
         assert chunk == p.chunk
         idx = torch.tensor(pgs, device=ro.device)
         got = pages[idx]                                  # [npc][2][Hh][P][d]

@@ -77,8 +77,9 @@ class Rollout:
         tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
         self.q_rot = torch.zeros(shape, dtype=tdt, device=self.device)
         self.out = torch.zeros(shape, dtype=tdt, device=self.device)
-        self.stored: Dict[int, tuple] = {}   # chunk -> (k bits, v bits) the store published
-        self.live: Dict[int, tuple] = {}     # slot -> (q, k, v bits, chunk) this round
+        # per layer: chunk -> (k bits, v bits) the store published; slot -> (q, k, v, chunk)
+        self.stored: Dict[int, Dict[int, tuple]] = {l: {} for l in range(self.layers)}
+        self.live: Dict[int, Dict[int, tuple]] = {l: {} for l in range(self.layers)}
 
     @property
     def round(self) -> int:
@@ -100,13 +101,13 @@ class Rollout:
         self.inputs = inputs
         tq, tk, tv = (to_device(x, c.dtype, self.device) for x in (q, k, v))
         self.pool.publish(layer, tq, tk, tv, self.q_rot)
-        self.live = {}
+        self.live[layer] = {}
         for p in lay:
             if p.slot is None:
                 continue
-            self.live[p.slot] = (q[p.slot], k[p.slot], v[p.slot], p.chunk)
+            self.live[layer][p.slot] = (q[p.slot], k[p.slot], v[p.slot], p.chunk)
             if p.kind == "store":
-                self.stored[p.chunk] = (k[p.slot], v[p.slot])
+                self.stored[layer][p.chunk] = (k[p.slot], v[p.slot])
         return inputs
 
     def attention(self, layer: int = 0, fill: float = float("nan")):
@@ -124,33 +125,33 @@ class Rollout:
         return O.rope_3d(x64, chunk, c.frames_per_chunk, c.grid_h, c.grid_w,
                          split=c.rope_split, base=c.rope_base)
 
-    def oracle_tensors(self, heads: Sequence[int]):
+    def oracle_tensors(self, heads: Sequence[int], layer: int = 0):
         """fp64 rotated q per live slot, rotated K and V per context chunk."""
         c, hs = self.cfg, list(heads)
         q_rot, keys, vals = {}, {}, {}
-        for s, (q, k, v, chunk) in self.live.items():
+        for s, (q, k, v, chunk) in self.live[layer].items():
             q_rot[s] = self._rope(to_f64(q, c.dtype)[:, hs], chunk)
         for p in self.layout():
             if p.slot is None:
-                kb, vb = self.stored[p.chunk]
+                kb, vb = self.stored[layer][p.chunk]
             else:
-                _, kb, vb, _ = self.live[p.slot]
+                _, kb, vb, _ = self.live[layer][p.slot]
             keys[p.chunk] = self._rope(to_f64(kb, c.dtype)[:, hs], p.chunk)
             vals[p.chunk] = to_f64(vb, c.dtype)[:, hs]
         return q_rot, keys, vals
 
-    def oracle_out(self, heads: Sequence[int], rows: Optional[np.ndarray] = None):
-        q_rot, keys, vals = self.oracle_tensors(heads)
+    def oracle_out(self, heads: Sequence[int], rows: Optional[np.ndarray] = None, layer: int = 0):
+        q_rot, keys, vals = self.oracle_tensors(heads, layer)
         return O.attention_slot_prefix(q_rot, keys, vals, self.layout(), rows=rows)
 
-    def oracle_out_bf16_operands(self, heads: Sequence[int], rows=None):
+    def oracle_out_bf16_operands(self, heads: Sequence[int], rows=None, layer: int = 0):
         """Oracle attention on operands rounded to the published bf16 format.
 
         The oracle rotates q and k in float64 and rounds them to bf16 itself
         (round_bf16), modelling the storage format of q_rot and the K pages;
         nothing here is read back from the GPU.
         """
-        q_rot, keys, vals = self.oracle_tensors(heads)
+        q_rot, keys, vals = self.oracle_tensors(heads, layer)
         q_rot = {s: O.round_bf16(x) for s, x in q_rot.items()}
         keys = {c: O.round_bf16(x) for c, x in keys.items()}
         return O.attention_slot_prefix(q_rot, keys, vals, self.layout(), rows=rows)
