@@ -9,29 +9,25 @@
 //
 // One CTA computes O = softmax(Q K^T / sqrt(d)) V for two 128-row query tiles
 // (q = 0, 1) of one (slot, head), sharing every K/V page it loads:
-//   warp 16 (one lane) TMA producer: Q0, Q1 once, then for every key tile (one
+//   warp 8 (one lane)  TMA producer: Q0, Q1 once, then for every key tile (one
 //                      128-token page, found through the page table) K and V
 //                      into a two-stage shared-memory ring (128-byte swizzle).
-//   warp 17 (one lane) tcgen05 issuer, in the order
+//   warp 9 (one lane)  tcgen05 issuer, in the order
 //                        S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ...
 //                      S_q = Q_q K^T goes to TMEM columns [128q, 128q+128);
-//                      PV_q reads P_q from TMEM (bf16 pairs written over S_q:
-//                      keys 0-63 in columns 0-31, keys 64-127 in columns 64-95)
-//                      and accumulates O_q in columns 256 + 128q. While the
-//                      softmax of tile q works on S_q(j+1), the tensor pipe runs
+//                      PV_q reads P_q from TMEM (the first 64 columns of S_q,
+//                      bf16 pairs) and accumulates O_q in columns 256 + 128q.
+//                      While softmax q works on S_q(j+1), the tensor pipe runs
 //                      the other tile's P*V and S (ping-pong).
-//   warps 0-15         softmax, four warpgroups: tile q = wg / 2, column half
-//                      hf = wg % 2. A query row (TMEM lane) is shared by two
-//                      warps, one per 64-column half: each takes the max of its
-//                      half, the two exchange it through shared memory (an
-//                      mbarrier of 64 arrivals, so every wait stays bounded),
-//                      then each computes its half of P, rounds it to bf16 into
-//                      TMEM, keeps its half of the row sum and owns its half of
-//                      O. O is rescaled only when the running max grows by more
-//                      than 2^8 (the exponentials stay <= 256 otherwise). The
-//                      epilogue adds the two half sums, divides, stages the bf16
-//                      half rows in the tile's (now idle) Q buffer and each warp
-//                      writes its 32 x 64 box with a TMA store that clips rows
+//   warps 0-3 / 4-7    softmax of tile 0 / tile 1: thread r owns query row r
+//                      (TMEM lane r); row max and sum are thread-local over its
+//                      128 columns; P is rounded to bf16 and stored back into
+//                      TMEM; O is rescaled in TMEM only when the running max
+//                      grows by more than 2^8 (the exponentials stay <= 256
+//                      otherwise), which is the only time softmax waits for the
+//                      previous P*V. The epilogue divides by the row sum, stages
+//                      the bf16 rows in the tile's (now idle) Q buffer and each
+//                      warp writes its 32 rows with a TMA store that clips rows
 //                      past C.
 // Every wait is bounded: on timeout the CTA records WF_ERR_TIMEOUT, the other
 // roles see the abort flag, in-flight copies and MMAs are drained and TMEM is
@@ -54,18 +50,17 @@ constexpr int kHD = 128;              // head dim
 constexpr uint32_t kHalf = 16384;     // one [128 rows][64 cols] bf16 swizzled block
 constexpr uint32_t kTile = 2 * kHalf; // [128][128] bf16
 constexpr int kPageCache = 1024;      // page ids cached in shared memory
-// Warpgroups 0-3 run the softmax (tile, column half); warpgroup 4 holds the
-// TMA producer (warp 16) and the MMA issuer (warp 17); warps 18-19 only hand
-// their registers over. Launched at 96 registers per thread (640 x 96 =
-// 61440), warpgroup 4 drops to 56 and the softmax warpgroups rise to 104:
-// 512 x 104 + 128 x 56 = 60416.
-constexpr int kThreads = 640;
-constexpr int kSoftmaxWarps = 16;
-constexpr int kProducerWarp = 16;
-constexpr int kMmaWarp = 17;
-constexpr uint32_t kRegsSoftmax = 104;
-constexpr uint32_t kRegsControl = 56;
-static_assert(512 * kRegsSoftmax + 128 * kRegsControl <= 640 * 96, "register split");
+// Warpgroups 0 and 1 run the softmax of tiles 0 and 1; warpgroup 2 holds the
+// TMA producer (warp 8) and the MMA issuer (warp 9); warps 10-11 only hand
+// their registers over. Launched at 168 registers per thread (384 x 168 =
+// 64512), warpgroup 2 drops to 64 and the softmax warpgroups rise to 216:
+// 256 x 216 + 128 x 64 = 63488.
+constexpr int kThreads = 384;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kRegsSoftmax = 216;
+constexpr uint32_t kRegsControl = 64;
+static_assert(256 * kRegsSoftmax + 128 * kRegsControl <= 384 * 168, "register split");
 constexpr long long kWaitLimit = 2000000000LL;  // ~1 s at 2 GHz
 
 // TMEM columns.
@@ -77,16 +72,14 @@ constexpr uint32_t kOffQ = 0;                       // Q0, Q1
 constexpr uint32_t kOffK = kOffQ + 2 * kTile;       // 2 stages
 constexpr uint32_t kOffV = kOffK + 2 * kTile;       // 2 stages
 constexpr uint32_t kOffBar = kOffV + 2 * kTile;
-constexpr int kNumBars = 24;
+constexpr int kNumBars = 16;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kOffXchg = kOffMisc + 64;                 // [2 parity][2 q][2 half][128] f32
-constexpr uint32_t kOffPages = kOffXchg + 2 * 2 * 2 * 128 * 4;
+constexpr uint32_t kOffPages = kOffMisc + 64;
 constexpr uint32_t kSmemBytes = kOffPages + kPageCache * 4 + 1024;   // + alignment slack
 
 enum Bar {
   kQFull = 0, kKFull0 = 1, kKEmpty0 = 3, kVFull0 = 5, kVEmpty0 = 7,
-  kSFull0 = 9, kPReady0 = 11, kPVDone0 = 13, kDrain = 15,
-  kXchg0 = 16   // 8 barriers: (tile q, TMEM lane quadrant) pairs of softmax warps
+  kSFull0 = 9, kPReady0 = 11, kPVDone0 = 13, kDrain = 15
 };
 
 struct Ctx {
@@ -197,10 +190,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
       *abort_flag = 0;
       for (int b = 0; b < kNumBars; ++b) {
-        uint32_t count = 1;
-        if (b == kPReady0 || b == kPReady0 + 1) count = 2 * kBM;   // both column halves
-        if (b >= kXchg0) count = 64;                               // the two warps of a pair
-        mbar_init(bars + b, count);
+        // p_ready: one elected arrival per softmax warp of the tile
+        const bool softmax_arrives = b == kPReady0 || b == kPReady0 + 1;
+        mbar_init(bars + b, softmax_arrives ? kBM / 32 : 1);
       }
       fence_barrier_init();
     }
@@ -223,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tiles = npos * p.npc;
   const int last_valid = p.C - (p.npc - 1) * p.P;   // keys in a chunk's last page
 
-  if (warp >= kSoftmaxWarps) {
+  if (warp >= 8) {
    setmaxnreg_dec<kRegsControl>();
    if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer --
@@ -286,10 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t aV = smem_u32(smem + kOffV + (j & 1) * kTile);
 #pragma unroll
         for (int k = 0; k < kBN / 16; ++k) {
-          // A = P_q from TMEM: 16 keys = 8 columns of bf16 pairs per step; keys
-          // 64-127 sit 64 columns further (each column half writes its own P).
-          mma_bf16_ts(tmem + kTmemO + q * 128,
-                      tmem + kTmemS + q * 128 + (k < 4 ? k * 8 : 64 + (k - 4) * 8),
+          // A = P_q from TMEM: 16 keys = 8 columns of bf16 pairs per step.
+          mma_bf16_ts(tmem + kTmemO + q * 128, tmem + kTmemS + q * 128 + k * 8,
                       make_desc_sw128(aV + k * 2048, kHalf, 1024), idPV,
                       (j > 0 || k > 0) ? 1u : 0u);
         }
@@ -330,69 +320,55 @@ __global__ void __launch_bounds__(kThreads, 1)
    }
   } else {
    setmaxnreg_inc<kRegsSoftmax>();
-   const int wg = warp >> 2;
-   const int q = wg >> 1, hf = wg & 1;
-   if (q == 0 || has_q1) {
+   if (warp < 4 || has_q1) {
     // ------------------------------------------------------------- softmax --
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;                      // query row == TMEM lane
-    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_addr + kTmemS + q * 128 + hf * 64;   // this half's S
-    const uint32_t tO = tmem + lane_addr + kTmemO + q * 128 + hf * 64;   // this half's O
-    float *xchg = reinterpret_cast<float *>(smem + kOffXchg);
-    const int xbar = kXchg0 + q * 4 + quad;
+    const int q = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;               // query row == TMEM lane
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + kTmemS + q * 128;
+    const uint32_t tO = tmem + lane_addr + kTmemO + q * 128;
     float m = -INFINITY, l = 0.0f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       ok = __all_sync(0xffffffffu, wait_bar(ctx, kSFull0 + q, j & 1));
-      uint32_t s[64];
-      float mx = -INFINITY;
-      if (ok) {
-        tc_fence_after();
-        tmem_ld32(tS, s);
-        tmem_ld32(tS + 32, s + 32);
-        tmem_ld_wait();
-        reg_fence32(s);
-        reg_fence32(s + 32);
-        const int valid = (j % p.npc == p.npc - 1) ? last_valid - hf * 64 : 64;
-        if (valid < 64) {
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[128];
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c >= valid) s[c] = __float_as_uint(-INFINITY);
-        }
-        // Max of this half: eight chains of three-input max, then a tree.
-        float m8[8];
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s + c * 32);
+      tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float a = max3(__uint_as_float(s[i]), __uint_as_float(s[i + 8]), __uint_as_float(s[i + 16]));
-          a = max3(a, __uint_as_float(s[i + 24]), __uint_as_float(s[i + 32]));
-          a = max3(a, __uint_as_float(s[i + 40]), __uint_as_float(s[i + 48]));
-          m8[i] = fmaxf(a, __uint_as_float(s[i + 56]));
-        }
-        mx = fmaxf(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], max3(m8[5], m8[6], m8[7])));
+      for (int c = 0; c < 4; ++c) reg_fence32(s + c * 32);
+
+      const int valid = (j % p.npc == p.npc - 1) ? last_valid : kBN;
+      if (valid < kBN) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) s[c] = __float_as_uint(-INFINITY);
       }
-      // Exchange the half maxima (and whether this warp is still running) with
-      // the partner warp; both halves then take the same decisions.
-      float *slot_self = xchg + (((j & 1) * 2 + q) * 2 + hf) * 128;
-      float *slot_other = xchg + (((j & 1) * 2 + q) * 2 + (hf ^ 1)) * 128;
-      slot_self[r] = ok ? mx : __int_as_float(0x7fc00000);   // NaN = partner stopped
-      mbar_arrive(bars + xbar);
-      ok = __all_sync(0xffffffffu, ok && wait_bar(ctx, xbar, j & 1));
-      if (!ok) break;
-      const float mo = slot_other[r];
-      ok = __all_sync(0xffffffffu, !isnan(mo));
-      if (!ok) break;
-      const float m_new = fmaxf(m, fmaxf(mx, mo) * p.scale_log2);
+      // Row max: eight independent chains of three-input max, then a tree.
+      float m8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float a = max3(__uint_as_float(s[i]), __uint_as_float(s[i + 8]), __uint_as_float(s[i + 16]));
+#pragma unroll
+        for (int b = 24; b < 120; b += 16)
+          a = max3(a, __uint_as_float(s[b + i]), __uint_as_float(s[b + 8 + i]));
+        m8[i] = fmaxf(a, __uint_as_float(s[120 + i]));
+      }
+      const float mx = fmaxf(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], max3(m8[5], m8[6], m8[7])));
+      const float m_new = fmaxf(m, mx * p.scale_log2);
       const bool rescale = m_new - m > 8.0f;             // always true on the first tile
       const float alpha = rescale ? ex2(m - m_new) : 1.0f;
       const float m_use = rescale ? m_new : m;
       // P = 2^(s * log2(e) / sqrt(d) - m) on the MUFU unit, the scale-subtract
       // and the row sums in packed f32x2 arithmetic; rounded to bf16 pairs and
-      // stored over the first 32 columns of this half's S.
+      // streamed back into the first 64 columns of S_q, 16 columns (32 keys) at
+      // a time.
       const uint64_t sc2 = f2(p.scale_log2, p.scale_log2), nm2 = f2(-m_use, -m_use);
       uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
+      for (int cc = 0; cc < 4; ++cc) {
         uint32_t pw[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
@@ -416,13 +392,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, wait_bar(ctx, kPVDone0 + q, (j - 1) & 1));
         if (!ok) break;
         tc_fence_after();
-        const uint64_t a2 = f2(alpha, alpha);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           tmem_ld32(tO + c * 32, o);
           tmem_ld_wait();
           reg_fence32(o);
+          const uint64_t a2 = f2(alpha, alpha);
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             const uint64_t v = fmul2(f2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
@@ -436,37 +412,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bars + kPReady0 + q);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + kPReady0 + q);
     }
-    // Epilogue: add the two half sums (one more exchange), wait for the last
-    // P*V, divide and store this half of the rows.
     if (ok && n_tiles > 0) {
       ok = __all_sync(0xffffffffu, wait_bar(ctx, kPVDone0 + q, (n_tiles - 1) & 1));
-    }
-    {
-      const int j = n_tiles;
-      float *slot_self = xchg + (((j & 1) * 2 + q) * 2 + hf) * 128;
-      float *slot_other = xchg + (((j & 1) * 2 + q) * 2 + (hf ^ 1)) * 128;
-      slot_self[r] = ok ? l : __int_as_float(0x7fc00000);
-      mbar_arrive(bars + xbar);
-      ok = __all_sync(0xffffffffu, ok && wait_bar(ctx, xbar, j & 1));
-      const float lo = ok ? slot_other[r] : 0.0f;
-      ok = __all_sync(0xffffffffu, ok && !isnan(lo));
-      l += lo;
     }
     if (ok && n_tiles > 0) {
       tc_fence_after();
       const float inv = 1.0f / l;
-      // Stage this half (64 columns = one 128-byte swizzled block of the output
-      // tensor map) in the tile's Q buffer, whose last reader, the final S MMA,
-      // has completed: 16-byte chunk c of row r lands at hf * 16 KB + r * 128 +
-      // ((c ^ (r & 7)) * 16), so each warp's 32 rows form one contiguous 4 KB
-      // box and the warp stores it itself.
-      uint8_t *stage = smem + kOffQ + q * kTile + hf * kHalf;
+      // Stage the bf16 rows in this tile's Q buffer (its last reader, the final
+      // S MMA, has completed) in the 128-byte swizzled layout of the output
+      // tensor map, whose box is 32 rows: 16-byte chunk c of row r in 64-column
+      // half kt lands at kt * 16 KB + r * 128 + ((c ^ (r & 7)) * 16), so each
+      // warp's 32 rows form one contiguous 4 KB box per half and the warp
+      // stores them itself (no cross-warp barrier).
+      uint8_t *stage = smem + kOffQ + q * kTile;
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
+      for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t o[32];
-        tmem_ld32(tO + c2 * 32, o);
+        tmem_ld32(tO + c4 * 32, o);
         tmem_ld_wait();
         reg_fence32(o);
         uint32_t w[16];
@@ -475,8 +440,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           w[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int c = c2 * 4 + i;                       // 16-byte chunk 0..7 of the half row
-          const uint32_t addr = smem_u32(stage + r * 128 + ((c ^ (r & 7)) << 4));
+          const int cc = c4 * 4 + i;                      // 16-byte chunk 0..15 of the row
+          const int kt = cc >> 3, c = cc & 7;
+          const uint32_t addr = smem_u32(stage + kt * kHalf + r * 128 + ((c ^ (r & 7)) << 4));
           asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[4 * i]),
                        "r"(w[4 * i + 1]), "r"(w[4 * i + 2]), "r"(w[4 * i + 3])
                        : "memory");
@@ -484,9 +450,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      const int wr = quad * 32;                           // this warp's first row in the tile
+      const int wr = (warp & 3) * 32;                     // this warp's first row in the tile
       if (lane == 0 && row0 + q * kBM + wr < p.C) {       // boxes wholly past C are skipped
-        tma_store_4d(&tout, stage + wr * 128, hf * 64, h, row0 + q * kBM + wr, slot);
+        tma_store_4d(&tout, stage + wr * 128, 0, h, row0 + q * kBM + wr, slot);
+        tma_store_4d(&tout, stage + kHalf + wr * 128, 64, h, row0 + q * kBM + wr, slot);
         tma_store_commit();
         tma_store_wait_all();
       }
