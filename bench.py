@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="wan13b_bf16")
+    ap.add_argument("--mask", choices=["wf", "rf"], default="wf",
+                    help="wf: M_WF chunk-causal mask; rf: bidirectional live window")
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -138,12 +140,15 @@ class ClockSampler:
 
 def unmasked_flops(layout, cfg):
     """4 * C * (keys visible to the slot) * d * heads summed over live slots:
-    QK^T and PV multiply-adds over unmasked (query, key) pairs only."""
+    QK^T and PV multiply-adds over unmasked (query, key) pairs only. Under the
+    WF mask a slot reads the context prefix up to its own entry; under RF the
+    whole context."""
     total = 0
     for idx, (kind, chunk, slot, tag, pages) in enumerate(layout):
         if slot is None:
             continue
-        total += 4 * cfg.chunk_tokens * (idx + 1) * cfg.chunk_tokens * cfg.head_dim * cfg.num_heads
+        nvis = len(layout) if cfg.mask == "rf" else idx + 1
+        total += 4 * cfg.chunk_tokens * nvis * cfg.chunk_tokens * cfg.head_dim * cfg.num_heads
     return total
 
 
@@ -245,7 +250,7 @@ def run_ours(args, ws, rank, local):
     import wf_inputs
     from chunk_causal_wavefront_b200 import KVPool, make_config
 
-    cfg = wf_inputs.CONFIGS[args.config]
+    cfg = wf_inputs.CONFIGS[args.config].replace(mask=args.mask)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
@@ -258,7 +263,7 @@ def run_ours(args, ws, rank, local):
                               page_tokens=cfg.page_tokens, num_layers=1, dtype=cfg.dtype,
                               rope=cfg.rope, frames_per_chunk=cfg.frames_per_chunk,
                               grid_h=cfg.grid_h, grid_w=cfg.grid_w, rope_split=cfg.rope_split,
-                              rope_base=cfg.rope_base, max_rounds=total_rounds),
+                              rope_base=cfg.rope_base, max_rounds=total_rounds, mask=cfg.mask),
                   device=dev, page_order=wf_inputs.draw_page_order(npages, cfg.seed + 1))
     shape = (cfg.num_slots, cfg.chunk_tokens, cfg.num_heads, cfg.head_dim)
     tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
@@ -464,7 +469,7 @@ def run_reference(args, ws, rank):
 
 
 def workload_config(cfg, n):
-    return {"workload": f"{cfg.name}: one layer-round, S={cfg.num_stages}+store, "
+    return {"workload": f"{cfg.name}{'' if cfg.mask == 'wf' else ' (RF mask)'}: one layer-round, S={cfg.num_stages}+store, "
                         f"C={cfg.chunk_tokens}, heads={cfg.num_heads}x{cfg.head_dim}, "
                         f"anchor={cfg.anchor_chunks}, history={cfg.history_chunks}, "
                         f"page={cfg.page_tokens}, steady state",

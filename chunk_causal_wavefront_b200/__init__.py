@@ -8,7 +8,8 @@ package is its Python binding.
 """
 from .wf import (LIB_PATH, WF_DTYPE_BF16, WF_DTYPE_F32, WF_ERR_BAD_PAGE, WF_ERR_CALL_ORDER,
                  WF_ERR_CUDA, WF_ERR_INVALID_ARG, WF_ERR_NOT_READY, WF_ERR_OUT_OF_PAGES,
-                 WF_ERR_TIMEOUT, WF_ERR_UNSUPPORTED, WF_OK, WF_ROPE_3D, WF_ROPE_OFF, WfError,
+                 WF_ERR_TIMEOUT, WF_ERR_UNSUPPORTED, WF_MASK_RF, WF_MASK_WF, WF_OK, WF_ROPE_3D,
+                 WF_ROPE_OFF, WfError,
                  WfPoolConfig, wf_status_string)
 from .pool import KVPool, make_config
 
@@ -16,5 +17,5 @@ __all__ = [
     "KVPool", "make_config", "WfError", "WfPoolConfig", "wf_status_string", "LIB_PATH",
     "WF_OK", "WF_ERR_INVALID_ARG", "WF_ERR_OUT_OF_PAGES", "WF_ERR_NOT_READY", "WF_ERR_BAD_PAGE",
     "WF_ERR_CALL_ORDER", "WF_ERR_CUDA", "WF_ERR_UNSUPPORTED", "WF_ERR_TIMEOUT",
-    "WF_DTYPE_BF16", "WF_DTYPE_F32", "WF_ROPE_OFF", "WF_ROPE_3D",
+    "WF_DTYPE_BF16", "WF_DTYPE_F32", "WF_ROPE_OFF", "WF_ROPE_3D", "WF_MASK_WF", "WF_MASK_RF",
 ]

@@ -62,6 +62,7 @@ wf_status validate(const wf_pool_config &c) {
   if (c.history_chunks < 0 || c.history_chunks > WF_MAX_HISTORY) return WF_ERR_INVALID_ARG;
   if (c.page_tokens < 1 || c.num_layers < 1 || c.max_rounds < 1) return WF_ERR_INVALID_ARG;
   if (c.num_pages < 0) return WF_ERR_INVALID_ARG;
+  if (c.mask_mode != WF_MASK_WF && c.mask_mode != WF_MASK_RF) return WF_ERR_INVALID_ARG;
   if (c.dtype == WF_DTYPE_BF16) {
     if (c.head_dim != 128 || c.page_tokens != 128) return WF_ERR_UNSUPPORTED;
   } else if (c.dtype == WF_DTYPE_F32) {
@@ -235,7 +236,9 @@ LiveSlots live_slots(const wf_pool *p) {
     l.slot[l.n] = q.slot;
     l.chunk[l.n] = q.chunk;
     l.tag[l.n] = q.tag;
-    l.npos[l.n] = static_cast<int32_t>(i) + 1;   // the prefix up to its own entry
+    // WF: the context prefix up to its own entry; RF: the whole context.
+    l.npos[l.n] = p->cfg.mask_mode == WF_MASK_RF ? static_cast<int32_t>(p->layout.size())
+                                                  : static_cast<int32_t>(i) + 1;
     ++l.n;
   }
   return l;

@@ -20,7 +20,7 @@ def make_config(*, num_stages: int, chunk_tokens: int, num_heads: int, head_dim:
                 dtype: str = "bf16", rope: int = 0, frames_per_chunk: int = 1, grid_h: int = 1,
                 grid_w: int = 1, rope_split: Sequence[int] = (0, 0, 0),
                 rope_base: float = 10000.0, max_rounds: int = 1024,
-                num_pages: int = 0) -> WfPoolConfig:
+                num_pages: int = 0, mask: str = "wf") -> WfPoolConfig:
     c = WfPoolConfig()
     c.num_stages, c.chunk_tokens, c.num_heads, c.head_dim = num_stages, chunk_tokens, num_heads, head_dim
     c.anchor_chunks, c.history_chunks, c.page_tokens = anchor_chunks, history_chunks, page_tokens
@@ -33,6 +33,7 @@ def make_config(*, num_stages: int, chunk_tokens: int, num_heads: int, head_dim:
     c.rope_base = rope_base
     c.max_rounds = max_rounds
     c.num_pages = num_pages
+    c.mask_mode = {"wf": _wf.WF_MASK_WF, "rf": _wf.WF_MASK_RF}[mask]
     return c
 
 

@@ -26,6 +26,8 @@ WF_DTYPE_BF16 = 0
 WF_DTYPE_F32 = 1
 WF_ROPE_OFF = 0
 WF_ROPE_3D = 1
+WF_MASK_WF = 0
+WF_MASK_RF = 1
 KIND_NAMES = {0: "anchor", 1: "history", 2: "store", 3: "slot"}
 
 EXPORTS = (
@@ -45,7 +47,7 @@ class WfPoolConfig(ctypes.Structure):
         ("frames_per_chunk", ctypes.c_int32), ("grid_h", ctypes.c_int32),
         ("grid_w", ctypes.c_int32), ("rope_split", ctypes.c_int32 * 3),
         ("rope_base", ctypes.c_float), ("max_rounds", ctypes.c_int32),
-        ("num_pages", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32), ("mask_mode", ctypes.c_int32),
     ]
 
 

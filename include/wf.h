@@ -61,6 +61,13 @@ typedef enum {
 
 enum { WF_DTYPE_BF16 = 0, WF_DTYPE_F32 = 1 };
 enum { WF_ROPE_OFF = 0, WF_ROPE_3D = 1 };
+/* Which (query slot, key slot) pairs are visible.
+ * WF: M_WF(s, j) = 1[j >= s] (Method section of the hyper.ai summary), plus
+ *     anchor and history; masked pairs are never computed.
+ * RF: every live slot sees every other (bidirectional live window), the
+ *     Rolling Forcing graph that the pages contrast WF with ("Contexto",
+ *     e-cogni article); also sees anchor and history. */
+enum { WF_MASK_WF = 0, WF_MASK_RF = 1 };
 
 /* Limits of this implementation. */
 #define WF_MAX_STAGES 16
@@ -83,6 +90,7 @@ typedef struct {
   float rope_base;         /* rotary base (10000) */
   int32_t max_rounds;      /* rounds the pool may run (sizes the t table) */
   int32_t num_pages;       /* physical pages per layer; 0 = the minimum */
+  int32_t mask_mode;       /* WF_MASK_WF (default, 0) or WF_MASK_RF */
 } wf_pool_config;
 
 typedef struct wf_pool wf_pool;
@@ -134,8 +142,9 @@ wf_status wf_publish_kv(wf_pool *pool, int32_t layer, const void *q, const void 
 /* Round attention for one layer (M_WF mask, full attention inside chunks):
  * for every live query slot s and head h,
  *     out[s] = softmax(q_rot[s] K_s^T / sqrt(d)) V_s
- * where K_s, V_s are the keys of the ordered-context prefix slot s may read
- * (anchor, history, store, slots S-1 .. s). Before reading, the kernel checks
+ * where K_s, V_s are the keys slot s may read: under WF_MASK_WF the
+ * ordered-context prefix (anchor, history, store, slots S-1 .. s), under
+ * WF_MASK_RF the whole context. Before reading, the kernel checks
  * every page's ready tag against the round's expected tag; any mismatch sets
  * WF_ERR_NOT_READY in the status word and the launch writes no output.
  *   q_rot : [S+1][C][heads][d] rotated queries (as written by wf_publish_kv);

@@ -92,29 +92,34 @@ def round_layout(S: int, A: int, H: int, k: int) -> List[Position]:
     return pos
 
 
-def visible_positions(layout: Sequence[Position], s: int) -> List[int]:
+def visible_positions(layout: Sequence[Position], s: int, mask: str = "wf") -> List[int]:
     """Indices of the context entries query slot s attends to.
 
-    M_WF(s, j) = 1[j >= s] over live slots j (the store counts as j = S), plus
-    the anchor and history, which every query slot sees (Method section).
+    mask="wf": M_WF(s, j) = 1[j >= s] over live slots j (the store counts as
+    j = S), plus the anchor and history, which every query slot sees (Method
+    section). mask="rf": the Rolling Forcing graph the pages contrast WF with
+    (e-cogni "Contexto"; Method section: WF removes RF's reverse refinement),
+    read here as bidirectional attention among all live slots: every query
+    slot sees the whole context.
     """
     out = []
     for idx, p in enumerate(layout):
-        if p.kind in ("anchor", "history"):
+        if mask == "rf" or p.kind in ("anchor", "history"):
             out.append(idx)
         elif p.slot >= s:
             out.append(idx)
     return out
 
 
-def unmasked_flops(S: int, A: int, H: int, k: int, C: int, heads: int, d: int) -> int:
+def unmasked_flops(S: int, A: int, H: int, k: int, C: int, heads: int, d: int,
+                   mask: str = "wf") -> int:
     """Multiply-add FLOPs of QK^T and PV over visible (query, key) pairs."""
     layout = round_layout(S, A, H, k)
     total = 0
     for p in layout:
         if p.slot is None:
             continue
-        nvis = len(visible_positions(layout, p.slot))
+        nvis = len(visible_positions(layout, p.slot, mask))
         total += 4 * C * (nvis * C) * d * heads
     return total
 
@@ -204,7 +209,8 @@ def attention_slot_prefix(q_rot: Dict[int, np.ndarray], keys: Dict[int, np.ndarr
                           vals: Dict[int, np.ndarray], layout: Sequence[Position],
                           scale: Optional[float] = None,
                           heads: Optional[Sequence[int]] = None,
-                          rows: Optional[np.ndarray] = None) -> Dict[int, np.ndarray]:
+                          rows: Optional[np.ndarray] = None,
+                          mask: str = "wf") -> Dict[int, np.ndarray]:
     """O_s = softmax(Q_s K^T / sqrt(d)) V over the keys slot s may read.
 
     q_rot[s]: [C][heads][d] rotated queries of live slot s (store = S).
@@ -217,7 +223,7 @@ def attention_slot_prefix(q_rot: Dict[int, np.ndarray], keys: Dict[int, np.ndarr
         if p.slot is None:
             continue
         s = p.slot
-        vis = visible_positions(layout, s)
+        vis = visible_positions(layout, s, mask)
         K = np.concatenate([keys[layout[i].chunk] for i in vis], axis=0)
         V = np.concatenate([vals[layout[i].chunk] for i in vis], axis=0)
         Q = q_rot[s] if rows is None else q_rot[s][rows]
@@ -233,13 +239,14 @@ def attention_slot_prefix(q_rot: Dict[int, np.ndarray], keys: Dict[int, np.ndarr
 
 def attention_dense_mask(q_rot: Dict[int, np.ndarray], keys: Dict[int, np.ndarray],
                          vals: Dict[int, np.ndarray], layout: Sequence[Position],
-                         scale: Optional[float] = None) -> Dict[int, np.ndarray]:
+                         scale: Optional[float] = None, mask: str = "wf") -> Dict[int, np.ndarray]:
     """Second formulation: one dense token x token mask for the whole round.
 
     All context tokens form one key sequence and all live query tokens one query
     sequence. A query token of chunk i_q sees a key token of chunk i_k iff
     i_k <= i_q: itself (full attention inside the chunk) and every cleaner,
-    older chunk in the context, never a newer one (no reverse edge).
+    older chunk in the context, never a newer one (no reverse edge). With
+    mask="rf" every query token sees every context token.
     """
     q_slots = [p for p in layout if p.slot is not None]
     Q = np.concatenate([q_rot[p.slot] for p in q_slots], axis=0)
@@ -247,12 +254,15 @@ def attention_dense_mask(q_rot: Dict[int, np.ndarray], keys: Dict[int, np.ndarra
     K = np.concatenate([keys[p.chunk] for p in layout], axis=0)
     V = np.concatenate([vals[p.chunk] for p in layout], axis=0)
     k_chunk = np.concatenate([np.full(keys[p.chunk].shape[0], p.chunk) for p in layout])
-    mask = k_chunk[None, :] <= q_chunk[:, None]
+    if mask == "rf":
+        visible = np.ones((q_chunk.size, k_chunk.size), dtype=bool)
+    else:
+        visible = k_chunk[None, :] <= q_chunk[:, None]
     d = Q.shape[-1]
     sc = (1.0 / math.sqrt(d)) if scale is None else scale
     O = np.zeros(Q.shape[:2] + (V.shape[-1],), dtype=np.float64)
     for h in range(Q.shape[1]):
-        O[:, h] = _softmax_attend(Q[:, h], K[:, h], V[:, h], sc, mask=mask)
+        O[:, h] = _softmax_attend(Q[:, h], K[:, h], V[:, h], sc, mask=visible)
     out, r = {}, 0
     for p in q_slots:
         n = q_rot[p.slot].shape[0]
@@ -261,7 +271,7 @@ def attention_dense_mask(q_rot: Dict[int, np.ndarray], keys: Dict[int, np.ndarra
     return out
 
 
-def attention_bruteforce(q_rot, keys, vals, layout, scale=None):
+def attention_bruteforce(q_rot, keys, vals, layout, scale=None, mask="wf"):
     """Third formulation, pure Python loops (tiny inputs only).
 
     For every live query slot s, head h and query token, walk the context and
@@ -281,7 +291,7 @@ def attention_bruteforce(q_rot, keys, vals, layout, scale=None):
             for n in range(C):
                 logits, vs = [], []
                 for e in layout:
-                    if e.slot is not None and e.slot < s:
+                    if mask == "wf" and e.slot is not None and e.slot < s:
                         continue                      # M_WF(s, j) = 0 for j < s
                     for m in range(keys[e.chunk].shape[0]):
                         logits.append(sum(float(Q[n, h, c]) * float(keys[e.chunk][m, h, c])

@@ -150,3 +150,19 @@ def test_null_pool_arguments():
     assert lib.wf_advance_round(None, None) == W.WF_ERR_INVALID_ARG
     assert lib.wf_pool_destroy(None) == W.WF_ERR_INVALID_ARG
     assert lib.wf_kv_pool_bytes(None, None) == W.WF_ERR_INVALID_ARG
+
+
+def test_mask_mode_validation():
+    cfg = wf_inputs.CONFIGS["wan13b_bf16"]
+    c = pool_config(cfg)
+    c.mask_mode = 2
+    with pytest.raises(W.WfError) as e:
+        W.wf_kv_pool_bytes(c)
+    assert e.value.status == W.WF_ERR_INVALID_ARG
+    # the page table does not depend on the mask
+    a = wfb.KVPool(pool_config(cfg, mask="wf"))
+    b = wfb.KVPool(pool_config(cfg, mask="rf"))
+    for _ in range(9):
+        assert a.layout() == b.layout()
+        a.advance()
+        b.advance()

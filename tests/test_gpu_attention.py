@@ -73,8 +73,9 @@ def _compare(ro: Rollout, heads, rows=None, gpu_operands=True, name="", layer=0)
                 assert err <= BF16_ABS, (s, rec)
 
 
-def test_tiny_f32_every_round():
-    cfg = wf_inputs.CONFIGS["tiny_f32"]
+@pytest.mark.parametrize("mask", ["wf", "rf"])
+def test_tiny_f32_every_round(mask):
+    cfg = wf_inputs.CONFIGS["tiny_f32"].replace(mask=mask)
     ro = Rollout(cfg, page_seed=0)
     for k in range(cfg.rounds + 3):
         ro.publish(0)
@@ -97,7 +98,10 @@ SMALL_BF16 = wf_inputs.CONFIGS["wan13b_bf16"].replace(
                        frames_per_chunk=3, grid_h=4, grid_w=11),
     SMALL_BF16.replace(num_stages=1, history_chunks=0, chunk_tokens=128, grid_h=8, grid_w=16),
     SMALL_BF16.replace(chunk_tokens=1, grid_h=1, grid_w=1),
-], ids=["S3_C300", "noanchor_C132", "S1_C128", "C1"])
+    SMALL_BF16.replace(mask="rf"),
+    SMALL_BF16.replace(mask="rf", anchor_chunks=0, history_chunks=1, chunk_tokens=3 * 4 * 11,
+                       frames_per_chunk=3, grid_h=4, grid_w=11),
+], ids=["S3_C300", "noanchor_C132", "S1_C128", "C1", "rf_S3_C300", "rf_noanchor_C132"])
 def test_bf16_every_round_small(cfg):
     ro = Rollout(cfg, page_seed=4)
     for k in range(cfg.steady_round() + 3):
@@ -133,9 +137,10 @@ def _sample_rows(C, n, seed):
     return np.array(sorted(rows))
 
 
-@pytest.mark.parametrize("name", ["wan13b_bf16", "wan13b_5step_bf16", "wan14b_bf16"])
+@pytest.mark.parametrize("name", ["wan13b_bf16", "wan13b_5step_bf16", "wan14b_bf16", "wan13b_bf16_rf"])
 def test_full_size_sampled(name):
-    cfg = wf_inputs.CONFIGS[name]
+    cfg = (wf_inputs.CONFIGS["wan13b_bf16"].replace(mask="rf") if name.endswith("_rf")
+           else wf_inputs.CONFIGS[name])
     ro = _steady(cfg)
     heads = sorted({0, cfg.num_heads // 2, cfg.num_heads - 1})
     rows = _sample_rows(cfg.chunk_tokens, 40, 1)

@@ -323,3 +323,45 @@ def test_round_bf16_matches_library_cast():
     # ties: 1 + 2^-8 is halfway between 1 and 1 + 2^-7 -> even (1.0)
     assert O.round_bf16(np.array([1.0 + 2 ** -8]))[0] == 1.0
     assert O.round_bf16(np.array([1.0 + 3 * 2 ** -8]))[0] == 1.0 + 2 ** -6
+
+
+# --- Rolling Forcing mask variant ------------------------------------------------
+
+@pytest.mark.parametrize("S,A,H", [(2, 1, 1), (3, 0, 2)])
+def test_rf_three_formulations_agree(S, A, H):
+    C, Hh, d = 3, 2, 4
+    for layout, q, kk, vv in _run_rounds(S, A, H, C, Hh, d, S + A + H + 3, rope=True):
+        o1 = O.attention_slot_prefix(q, kk, vv, layout, mask="rf")
+        o2 = O.attention_dense_mask(q, kk, vv, layout, mask="rf")
+        o3 = O.attention_bruteforce(q, kk, vv, layout, mask="rf")
+        for s in o1:
+            np.testing.assert_allclose(o1[s], o2[s], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(o1[s], o3[s], rtol=0, atol=1e-12)
+
+
+def test_rf_has_reverse_edges_and_wf_does_not():
+    # Under RF a cleaner slot reads noisier live slots; under WF it never does.
+    S, A, H, C, Hh, d = 4, 1, 2, 5, 2, 8
+    layout, q, kk, vv = _run_rounds(S, A, H, C, Hh, d, 9)[-1]
+    j = 1
+    chunk_j = [p.chunk for p in layout if p.slot == j][0]
+    kk2 = dict(kk)
+    kk2[chunk_j] = kk[chunk_j] + 2.0 * _rand(kk[chunk_j].shape, 3)
+    for mask, cleaner_changes in (("rf", True), ("wf", False)):
+        base = O.attention_slot_prefix(q, kk, vv, layout, mask=mask)
+        pert = O.attention_slot_prefix(q, kk2, vv, layout, mask=mask)
+        for s in base:
+            if s > j:
+                assert (np.abs(pert[s] - base[s]).max() > 1e-3) == cleaner_changes, (mask, s)
+    # with one live slot the two graphs coincide
+    layout0, q0, k0, v0 = _run_rounds(S, A, H, C, Hh, d, 1)[0]
+    a = O.attention_slot_prefix(q0, k0, v0, layout0, mask="rf")[0]
+    b = O.attention_slot_prefix(q0, k0, v0, layout0, mask="wf")[0]
+    np.testing.assert_array_equal(a, b)
+
+
+def test_rf_work_closed_form():
+    # RF: every live slot reads the whole context of A + H + S + 1 chunks.
+    S, A, H = 4, 1, 2
+    k = S + A + H + 1
+    assert O.unmasked_flops(S, A, H, k, 7, 2, 8, "rf") == 4 * 7 * 7 * 8 * 2 * (S + 1) * (A + H + S + 1)

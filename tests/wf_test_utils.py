@@ -26,7 +26,7 @@ def pool_config(cfg: WorkloadConfig, **over):
               num_layers=cfg.num_layers, dtype=cfg.dtype, rope=cfg.rope,
               frames_per_chunk=cfg.frames_per_chunk, grid_h=cfg.grid_h, grid_w=cfg.grid_w,
               rope_split=cfg.rope_split if cfg.rope else (0, 0, 0), rope_base=cfg.rope_base,
-              max_rounds=max(cfg.rounds + 1, 16), num_pages=0)
+              max_rounds=max(cfg.rounds + 1, 16), num_pages=0, mask=cfg.mask)
     kw.update(over)
     return make_config(**kw)
 
@@ -142,7 +142,8 @@ class Rollout:
 
     def oracle_out(self, heads: Sequence[int], rows: Optional[np.ndarray] = None, layer: int = 0):
         q_rot, keys, vals = self.oracle_tensors(heads, layer)
-        return O.attention_slot_prefix(q_rot, keys, vals, self.layout(), rows=rows)
+        return O.attention_slot_prefix(q_rot, keys, vals, self.layout(), rows=rows,
+                                       mask=self.cfg.mask)
 
     def oracle_out_bf16_operands(self, heads: Sequence[int], rows=None, layer: int = 0):
         """Oracle attention on operands rounded to the published bf16 format.
@@ -154,7 +155,8 @@ class Rollout:
         q_rot, keys, vals = self.oracle_tensors(heads, layer)
         q_rot = {s: O.round_bf16(x) for s, x in q_rot.items()}
         keys = {c: O.round_bf16(x) for c, x in keys.items()}
-        return O.attention_slot_prefix(q_rot, keys, vals, self.layout(), rows=rows)
+        return O.attention_slot_prefix(q_rot, keys, vals, self.layout(), rows=rows,
+                                       mask=self.cfg.mask)
 
     def close(self):
         self.pool.close()

@@ -51,6 +51,7 @@ class WorkloadConfig:
     k_outlier_scale: float = 1.0  # by this power of two
     rounds: int = 1               # rounds run by the workload
     seed: int = 0
+    mask: str = "wf"              # "wf" (M_WF) or "rf" (bidirectional live window)
 
     @property
     def pages_per_chunk(self) -> int:
