@@ -7,20 +7,51 @@
 // assigns to each live slot; the ready signal is a per-page tag.
 //
 // One launch covers every live slot of the round (grid row = slot). A thread
-// owns one 16-byte vector column (8 bf16 or 4 fp32 values = 4 or 2 rotary
-// pairs) of the [C][heads][d] token rows and walks the block's tokens: it
-// loads q, k and v with streaming 16-byte loads, rotates q and k in fp32 with
-// (cos, sin) tables computed on the host in fp64, rounds once to the storage
-// type and issues 16-byte stores to q_rot and to the K and V pages.
-// Consecutive threads cover consecutive vectors of a token row, so loads are
-// fully coalesced; a warp's page stores cover two contiguous 256-byte head
-// rows. HBM-bound: 3 reads + 3 writes of every element.
+// handles 16-byte vectors (8 bf16 or 4 fp32 values = 4 or 2 rotary pairs) of
+// (slot, token, head) rows, two per iteration: it loads q, k and v with
+// streaming 16-byte loads,
+// rotates q and k in fp32 with (cos, sin) tables computed on the host in fp64,
+// rounds once to the storage type and issues 16-byte stores to q_rot and to
+// the K and V pages. Consecutive threads cover consecutive 16-byte vectors of
+// the [C][heads][d] input rows, so loads are fully coalesced; a warp's page
+// stores cover two contiguous 256-byte head rows. HBM-bound: 3 reads + 3
+// writes of every element.
 #include <cuda_bf16.h>
 
 #include "wf_internal.h"
 
 namespace wf {
 namespace {
+
+// Division by a runtime-invariant divisor d (1 <= d < 2^31) for dividends
+// n < 2^31 with one multiply-high and a shift (Granlund and Montgomery,
+// "Division by Invariant Integers using Multiplication", 1994): with
+// p = 31 + ceil(log2 d) and m = ceil(2^p / d), floor(n / d) = (n * m) >> p,
+// exact because m - 2^p / d < 1 keeps the error below 1 / d.
+struct FastDiv {
+  uint32_t d, m, shift;   // shift = p - 32 (d >= 2); d == 1 is the identity
+  __host__ __device__ FastDiv() : d(1), m(0), shift(0) {}
+  __host__ explicit FastDiv(uint32_t div) : d(div), m(0), shift(0) {
+    if (d > 1) {
+      uint32_t l = 0;
+      while ((uint64_t(1) << l) < d) ++l;                 // ceil(log2 d)
+      const uint64_t p2 = uint64_t(1) << (31 + l);
+      m = static_cast<uint32_t>((p2 + d - 1) / d);
+      shift = 31 + l - 32;
+    }
+  }
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    return d == 1 ? n : (__umulhi(n, m) >> shift);
+  }
+  __device__ __forceinline__ void divmod(uint32_t n, uint32_t &q, uint32_t &r) const {
+    q = div(n);
+    r = n - q * d;
+  }
+};
+
+struct PublishDivs {
+  FastDiv vpt, vpr, P, hw, gw, tail_rows, Hh;
+};
 
 template <typename T> struct Vec;
 template <> struct Vec<__nv_bfloat16> { static constexpr int N = 8; };
@@ -78,113 +109,111 @@ __device__ __forceinline__ void rope_vec(float *x, int dim0, int tpos, int ypos,
   }
 }
 
-constexpr int kTok = 16;   // tokens per block
+// Physical page holding page j of live slot li's chunk (-1 if the table is bad).
+__device__ __forceinline__ int slot_page(const PublishParams &p, int pos, int j) {
+  const int phys = pos < 0 ? -1 : __ldg(p.table + kTabPages + pos * p.npc + j);
+  return (phys < 0 || phys >= p.num_pages) ? -1 : phys;
+}
 
-// Grid: (token blocks + tail blocks, live slots); block = one thread per
-// 16-byte vector column (head, vector) of a token row, looping over columns
-// when a row has more vectors than the block has threads. A block first puts
-// its tokens' rotary positions and page rows in shared memory, so the inner
-// loop has no integer division: per token and column it issues three
-// streaming 16-byte loads (two tokens at a time), rotates q and k in fp32,
-// rounds once and issues three 16-byte stores. Tail blocks zero the rows past
-// C in the chunk's last page.
+// One main-part vector: rotate q and k, write q_rot and the K/V page rows.
 template <typename T>
-__global__ void __launch_bounds__(640) publish_kernel(const PublishParams p, int main_blocks) {
+__device__ __forceinline__ void publish_vector(const PublishParams &p, const PublishDivs &dv,
+                                               int li, int pos, int n, int h, int e,
+                                               const uint4 &qv, const uint4 &kv,
+                                               const uint4 &vv, size_t src) {
   constexpr int N = Vec<T>::N;
-  __shared__ int s_pos[3][kTok];       // t, y, x of the block's tokens
-  __shared__ int s_page[kTok];         // physical page of each token (-1: bad table entry)
-  __shared__ int s_row[kTok];          // row of each token inside its page
+  float q[N], k[N];
+  unpack(qv, q, T());
+  unpack(kv, k, T());
+  if (p.rope) {
+    // n = f * (gh * gw) + y * gw + x: frame f of the chunk, row y, column x
+    uint32_t f, yx, y, x;
+    dv.hw.divmod(n, f, yx);
+    dv.gw.divmod(yx, y, x);
+    const int tpos = p.F * p.live.chunk[li] + static_cast<int>(f);
+    rope_vec<N>(q, e * N, tpos, static_cast<int>(y), static_cast<int>(x), p);
+    rope_vec<N>(k, e * N, tpos, static_cast<int>(y), static_cast<int>(x), p);
+  }
+  *reinterpret_cast<uint4 *>(static_cast<T *>(p.q_rot) + src) = pack(q, T());
+  uint32_t ju, rowu;
+  dv.P.divmod(n, ju, rowu);
+  const int j = static_cast<int>(ju), row = static_cast<int>(rowu);
+  const int phys = slot_page(p, pos, j);
+  if (phys < 0) {
+    record_status(p.status, WF_ERR_BAD_PAGE);
+    return;
+  }
+  const size_t page_elems = static_cast<size_t>(2) * p.Hh * p.P * p.d;
+  T *kdst = reinterpret_cast<T *>(p.pages) + phys * page_elems +
+            (static_cast<size_t>(h) * p.P + row) * p.d + e * N;
+  T *vdst = kdst + static_cast<size_t>(p.Hh) * p.P * p.d;
+  *reinterpret_cast<uint4 *>(kdst) = pack(k, T());
+  *reinterpret_cast<uint4 *>(vdst) = vv;
+  if (row == 0 && h == 0 && e == 0) p.tags[phys] = p.live.tag[li];
+}
+
+// Grid: (blocks, live slots). Each thread walks its slot's vectors with a
+// grid stride, two at a time so that six 16-byte loads are in flight before
+// the first one is used. Vector v < C * heads * d/N is (token n, head h,
+// vector e) of the [C][heads][d] rows; the remaining vectors zero the rows
+// past C in the chunk's last page (K then V, head-major, row, vector).
+template <typename T>
+__global__ void __launch_bounds__(256) publish_kernel(const PublishParams p, const PublishDivs dv) {
+  constexpr int N = Vec<T>::N;
   const int li = blockIdx.y;
   const int slot = p.live.slot[li];
   const int pos = __ldg(p.table + kTabSlotPos + slot);
   const int vpr = p.d / N;                                   // vectors per head row
   const int vpt = p.Hh * vpr;                                // vectors per token
-  const size_t kv_elems = static_cast<size_t>(p.Hh) * p.P * p.d;   // K -> V distance
-  const size_t page_elems = 2 * kv_elems;
-  T *pages = reinterpret_cast<T *>(p.pages);
+  const int main_n = p.C * vpt;
+  const int tail_rows = p.npc * p.P - p.C;
+  const int total = main_n + 2 * p.Hh * tail_rows * vpr;
+  const size_t slot_off = static_cast<size_t>(slot) * p.C * p.Hh * p.d;
+  const T *qs = static_cast<const T *>(p.q) + slot_off;
+  const T *ks = static_cast<const T *>(p.k) + slot_off;
+  const T *vs = static_cast<const T *>(p.v) + slot_off;
+  const int stride = gridDim.x * blockDim.x;
 
-  if (blockIdx.x < main_blocks) {
-    const int n0 = blockIdx.x * kTok;
-    const int ntok = min(kTok, p.C - n0);
-    if (threadIdx.x < ntok) {
-      const int n = n0 + threadIdx.x;
-      if (p.rope) {
-        const int hw = p.gh * p.gw;
-        s_pos[0][threadIdx.x] = p.F * p.live.chunk[li] + n / hw;
-        s_pos[1][threadIdx.x] = (n / p.gw) % p.gh;
-        s_pos[2][threadIdx.x] = n % p.gw;
-      }
-      const int j = n / p.P, row = n - j * p.P;
-      const int phys = pos < 0 ? -1 : __ldg(p.table + kTabPages + pos * p.npc + j);
-      s_row[threadIdx.x] = row;
-      if (phys < 0 || phys >= p.num_pages) {
-        record_status(p.status, WF_ERR_BAD_PAGE);
-        s_page[threadIdx.x] = -1;
-      } else {
-        s_page[threadIdx.x] = phys;
-        if (row == 0) p.tags[phys] = p.live.tag[li];
-      }
+  for (int v0 = blockIdx.x * blockDim.x + threadIdx.x; v0 < total; v0 += 2 * stride) {
+    const int v1 = v0 + stride;
+    const bool m0 = v0 < main_n, m1 = v1 < main_n;
+    uint4 q0, k0, w0, q1, k1, w1;
+    if (m0) {
+      q0 = ld_stream(qs + static_cast<size_t>(v0) * N);
+      k0 = ld_stream(ks + static_cast<size_t>(v0) * N);
+      w0 = ld_stream(vs + static_cast<size_t>(v0) * N);
     }
-    __syncthreads();
-    const size_t slot_off = static_cast<size_t>(slot) * p.C * p.Hh * p.d;
-    for (int col = threadIdx.x; col < vpt; col += blockDim.x) {
-      const int h = col / vpr, e = col - h * vpr;
-      const size_t col_off = static_cast<size_t>(h) * p.d + e * N;   // inside a token row
-      const size_t page_col = static_cast<size_t>(h) * p.P * p.d + e * N;
-      for (int i = 0; i < ntok; i += 2) {
-        const bool two = i + 1 < ntok;
-        const size_t src0 = slot_off + static_cast<size_t>(n0 + i) * p.Hh * p.d + col_off;
-        const size_t src1 = src0 + static_cast<size_t>(p.Hh) * p.d;
-        const uint4 q0 = ld_stream(static_cast<const T *>(p.q) + src0);
-        const uint4 k0 = ld_stream(static_cast<const T *>(p.k) + src0);
-        const uint4 v0 = ld_stream(static_cast<const T *>(p.v) + src0);
-        uint4 q1 = make_uint4(0, 0, 0, 0), k1 = q1, v1 = q1;
-        if (two) {
-          q1 = ld_stream(static_cast<const T *>(p.q) + src1);
-          k1 = ld_stream(static_cast<const T *>(p.k) + src1);
-          v1 = ld_stream(static_cast<const T *>(p.v) + src1);
-        }
+    if (m1) {
+      q1 = ld_stream(qs + static_cast<size_t>(v1) * N);
+      k1 = ld_stream(ks + static_cast<size_t>(v1) * N);
+      w1 = ld_stream(vs + static_cast<size_t>(v1) * N);
+    }
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          if (u == 1 && !two) break;
-          const int t = i + u;
-          float q[N], k[N];
-          unpack(u ? q1 : q0, q, T());
-          unpack(u ? k1 : k0, k, T());
-          if (p.rope) {
-            rope_vec<N>(q, e * N, s_pos[0][t], s_pos[1][t], s_pos[2][t], p);
-            rope_vec<N>(k, e * N, s_pos[0][t], s_pos[1][t], s_pos[2][t], p);
-          }
-          *reinterpret_cast<uint4 *>(static_cast<T *>(p.q_rot) + (u ? src1 : src0)) = pack(q, T());
-          const int phys = s_page[t];
-          if (phys < 0) continue;
-          T *kdst = pages + phys * page_elems + page_col + static_cast<size_t>(s_row[t]) * p.d;
-          *reinterpret_cast<uint4 *>(kdst) = pack(k, T());
-          *reinterpret_cast<uint4 *>(kdst + kv_elems) = u ? v1 : v0;
+    for (int u = 0; u < 2; ++u) {
+      const int v = u ? v1 : v0;
+      if (v >= total) break;
+      if (u ? m1 : m0) {
+        uint32_t n, rem, h, e;
+        dv.vpt.divmod(v, n, rem);
+        dv.vpr.divmod(rem, h, e);
+        publish_vector<T>(p, dv, li, pos, n, h, e, u ? q1 : q0, u ? k1 : k0, u ? w1 : w0,
+                          slot_off + static_cast<size_t>(v) * N);
+      } else {
+        uint32_t r1, e, r2, rr, kv, h;
+        dv.vpr.divmod(v - main_n, r1, e);
+        dv.tail_rows.divmod(r1, r2, rr);
+        dv.Hh.divmod(r2, kv, h);
+        const int row = p.P - tail_rows + static_cast<int>(rr);
+        const int phys = slot_page(p, pos, p.npc - 1);
+        if (phys < 0) {
+          record_status(p.status, WF_ERR_BAD_PAGE);
+          continue;
         }
+        T *dst = reinterpret_cast<T *>(p.pages) +
+                 phys * (static_cast<size_t>(2) * p.Hh * p.P * p.d) +
+                 ((static_cast<size_t>(kv) * p.Hh + h) * p.P + row) * p.d + e * N;
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
       }
-    }
-  } else {
-    // Zero the rows past C in the chunk's last page: (K|V, head, row, vector).
-    const int tail_rows = p.npc * p.P - p.C;
-    const int total = 2 * p.Hh * tail_rows * vpr;
-    const int phys = pos < 0 ? -1 : __ldg(p.table + kTabPages + pos * p.npc + (p.npc - 1));
-    if (phys < 0 || phys >= p.num_pages) {
-      if (threadIdx.x == 0) record_status(p.status, WF_ERR_BAD_PAGE);
-      return;
-    }
-    const int tb = blockIdx.x - main_blocks, ntb = gridDim.x - main_blocks;
-    for (int v = tb * blockDim.x + threadIdx.x; v < total; v += ntb * blockDim.x) {
-      int r = v;
-      const int e = r % vpr;
-      r /= vpr;
-      const int row = p.P - tail_rows + r % tail_rows;
-      r /= tail_rows;
-      const int h = r % p.Hh;
-      const int kv = r / p.Hh;
-      T *dst = pages + phys * page_elems + kv * kv_elems +
-               (static_cast<size_t>(h) * p.P + row) * p.d + e * N;
-      *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
     }
   }
 }
@@ -193,14 +222,29 @@ template <typename T>
 cudaError_t launch(const PublishParams &p, cudaStream_t st) {
   if (p.live.n == 0) return cudaSuccess;
   constexpr int N = Vec<T>::N;
-  const int vpt = p.Hh * (p.d / N);
-  const int threads = vpt >= 640 ? 640 : ((vpt + 31) / 32) * 32;
-  const int main_blocks = (p.C + kTok - 1) / kTok;
-  const int64_t tail_vecs = 2LL * p.Hh * (p.npc * p.P - p.C) * (p.d / N);
-  const int tail_blocks = tail_vecs == 0 ? 0 : static_cast<int>((tail_vecs + threads - 1) / threads);
-  const int64_t per_slot = static_cast<int64_t>(p.C) * vpt + tail_vecs;
+  const int64_t vpr = p.d / N;
+  const int64_t per_slot = static_cast<int64_t>(p.C) * p.Hh * vpr +
+                           2LL * p.Hh * (p.npc * p.P - p.C) * vpr;
   if (per_slot >= (int64_t(1) << 30)) return cudaErrorInvalidValue;   // int32 vector indices
-  publish_kernel<T><<<dim3(main_blocks + tail_blocks, p.live.n), threads, 0, st>>>(p, main_blocks);
+  int sms = 148, dev = 0, per_sm = 4;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, publish_kernel<T>, 256, 0);
+  PublishDivs dv;
+  dv.vpt = FastDiv(static_cast<uint32_t>(p.Hh * (p.d / N)));
+  dv.vpr = FastDiv(static_cast<uint32_t>(p.d / N));
+  dv.P = FastDiv(static_cast<uint32_t>(p.P));
+  dv.hw = FastDiv(static_cast<uint32_t>(p.gh * p.gw));
+  dv.gw = FastDiv(static_cast<uint32_t>(p.gw));
+  dv.tail_rows = FastDiv(static_cast<uint32_t>(p.npc * p.P - p.C > 0 ? p.npc * p.P - p.C : 1));
+  dv.Hh = FastDiv(static_cast<uint32_t>(p.Hh));
+  if (per_sm < 1) per_sm = 1;
+  // One wave: every resident block slot of the GPU, spread over the live slots.
+  int64_t bx = (static_cast<int64_t>(sms) * per_sm) / p.live.n;
+  const int64_t need = (per_slot + 511) / 512;            // two vectors per thread
+  if (bx > need) bx = need;
+  if (bx < 1) bx = 1;
+  publish_kernel<T><<<dim3(static_cast<unsigned>(bx), static_cast<unsigned>(p.live.n)), 256, 0, st>>>(p, dv);
   return cudaGetLastError();
 }
 
