@@ -53,13 +53,13 @@ constexpr int kPageCache = 1024;      // page ids cached in shared memory
 // Warpgroups 0 and 1 run the softmax of tiles 0 and 1; warpgroup 2 holds the
 // TMA producer (warp 8) and the MMA issuer (warp 9); warps 10-11 only hand
 // their registers over. Launched at 168 registers per thread (384 x 168 =
-// 64512), warpgroup 2 drops to 64 and the softmax warpgroups rise to 216:
-// 256 x 216 + 128 x 64 = 63488.
+// 64512), warpgroup 2 moves to 96 and the softmax warpgroups to 200:
+// 256 x 200 + 128 x 96 = 63488.
 constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr uint32_t kRegsSoftmax = 216;
-constexpr uint32_t kRegsControl = 64;
+constexpr uint32_t kRegsSoftmax = 200;
+constexpr uint32_t kRegsControl = 96;
 static_assert(256 * kRegsSoftmax + 128 * kRegsControl <= 384 * 168, "register split");
 constexpr long long kWaitLimit = 2000000000LL;  // ~1 s at 2 GHz
 
@@ -148,6 +148,30 @@ __device__ __forceinline__ void reg_fence32(uint32_t *r) {
   WF_REG_FENCE8(r, 24);
 }
 
+// S_q = Q_q K(stage)^T: 8 k-steps of 16 along d; Q and K are [128][128] bf16
+// tiles stored as two 64-column 128-byte-swizzled halves.
+__device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_lo, uint32_t k_lo,
+                                        uint32_t hi) {
+  constexpr uint32_t idS = make_idesc_bf16(kBM, kBN, false);
+#pragma unroll
+  for (int k = 0; k < kHD / 16; ++k) {
+    const uint32_t off = ((k >> 2) * kHalf + (k & 3) * 32) >> 4;
+    mma_bf16_ss2(tmem_s, q_lo + off, k_lo + off, hi, idS, k > 0);
+  }
+}
+
+// O_q (+)= P_q V(stage): 8 k-steps of 16 keys; P_q is read from TMEM (8
+// columns of bf16 pairs per step), V is MN-major in shared memory.
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_lo,
+                                         uint32_t hi, bool accumulate_first) {
+  constexpr uint32_t idPV = make_idesc_bf16(kBM, kHD, true);
+#pragma unroll
+  for (int k = 0; k < kBN / 16; ++k) {
+    mma_bf16_ts2(tmem_o, tmem_p + k * 8, v_lo + ((k * 2048) >> 4), hi, idPV,
+                 (accumulate_first || k > 0) ? 1u : 0u);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bf16_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tq,
                      const __grid_constant__ CUtensorMap tkv,
@@ -231,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(sQ + kTile, &tq, bars + kQFull, 0, h, row0 + kBM, slot);
         tma_load_4d(sQ + kTile + kHalf, &tq, bars + kQFull, 64, h, row0 + kBM, slot);
       }
-      int nk[2] = {0, 0}, nv[2] = {0, 0};
+      int nk0 = 0, nk1 = 0, nv0 = 0, nv1 = 0;   // loads issued per stage
       for (int j = 0; j < n_tiles; ++j) {
         const int stg = j & 1;
         const uint32_t ph = (j >> 1) & 1;
@@ -244,74 +268,67 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(bars + kKFull0 + stg, kTile);
         tma_load_2d(sK, &tkv, bars + kKFull0 + stg, 0, rowk);
         tma_load_2d(sK + kHalf, &tkv, bars + kKFull0 + stg, 64, rowk);
-        ++nk[stg];
+        if (stg) ++nk1; else ++nk0;
         if (!wait_bar(ctx, kVEmpty0 + stg, ph ^ 1)) break;
         mbar_arrive_expect_tx(bars + kVFull0 + stg, kTile);
         tma_load_2d(sV, &tkv, bars + kVFull0 + stg, 0, rowv);
         tma_load_2d(sV + kHalf, &tkv, bars + kVFull0 + stg, 64, rowv);
-        ++nv[stg];
+        if (stg) ++nv1; else ++nv0;
       }
       // Drain: every load this thread issued has landed before the CTA exits.
-      for (int s = 0; s < 2; ++s) {
-        if (nk[s]) drain_wait(ctx, kKFull0 + s, (nk[s] - 1) & 1);
-        if (nv[s]) drain_wait(ctx, kVFull0 + s, (nv[s] - 1) & 1);
-      }
+      if (nk0) drain_wait(ctx, kKFull0, (nk0 - 1) & 1);
+      if (nk1) drain_wait(ctx, kKFull0 + 1, (nk1 - 1) & 1);
+      if (nv0) drain_wait(ctx, kVFull0, (nv0 - 1) & 1);
+      if (nv1) drain_wait(ctx, kVFull0 + 1, (nv1 - 1) & 1);
       drain_wait(ctx, kQFull, 0);
     }
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- MMA issuer --
     if (lane == 0) {
-      constexpr uint32_t idS = make_idesc_bf16(kBM, kBN, false);
-      constexpr uint32_t idPV = make_idesc_bf16(kBM, kHD, true);
-      const uint32_t aQ = smem_u32(smem + kOffQ);
-      auto issue_s = [&](int q, int j) {
-        const uint32_t aK = smem_u32(smem + kOffK + (j & 1) * kTile);
-#pragma unroll
-        for (int k = 0; k < kHD / 16; ++k) {
-          const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
-          mma_bf16_ss(tmem + kTmemS + q * 128, make_desc_sw128(aQ + q * kTile + off, 16, 1024),
-                      make_desc_sw128(aK + off, 16, 1024), idS, k > 0);
-        }
-        mma_commit(bars + kSFull0 + q);
-      };
-      auto issue_pv = [&](int q, int j) {
-        const uint32_t aV = smem_u32(smem + kOffV + (j & 1) * kTile);
-#pragma unroll
-        for (int k = 0; k < kBN / 16; ++k) {
-          // A = P_q from TMEM: 16 keys = 8 columns of bf16 pairs per step.
-          mma_bf16_ts(tmem + kTmemO + q * 128, tmem + kTmemS + q * 128 + k * 8,
-                      make_desc_sw128(aV + k * 2048, kHalf, 1024), idPV,
-                      (j > 0 || k > 0) ? 1u : 0u);
-        }
-        mma_commit(bars + kPVDone0 + q);
-      };
+      // Descriptor words: the high word (stride 1 KB, version, swizzle) is the
+      // same for Q, K and V; a k-step or a stage only moves the low word.
+      const uint32_t hi = desc_hi_sw128(1024);
+      const uint32_t q_lo = desc_lo_sw128(smem_u32(smem + kOffQ), 16);
+      const uint32_t k_lo = desc_lo_sw128(smem_u32(smem + kOffK), 16);
+      const uint32_t v_lo = desc_lo_sw128(smem_u32(smem + kOffV), kHalf);
+      constexpr uint32_t kTileStep = kTile >> 4;
       bool ok = wait_bar(ctx, kQFull, 0) && wait_bar(ctx, kKFull0, 0);
       if (ok) {
         tc_fence_after();
-        issue_s(0, 0);
-        if (has_q1) issue_s(1, 0);
+        issue_s(tmem + kTmemS, q_lo, k_lo, hi);
+        mma_commit(bars + kSFull0);
+        if (has_q1) {
+          issue_s(tmem + kTmemS + 128, q_lo + kTileStep, k_lo, hi);
+          mma_commit(bars + kSFull0 + 1);
+        }
         mma_commit(bars + kKEmpty0);
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int stg = j & 1;
+        const int stg = j & 1, nstg = (j + 1) & 1;
         const bool more = j + 1 < n_tiles;
         if (!wait_bar(ctx, kVFull0 + stg, (j >> 1) & 1)) break;
         if (!wait_bar(ctx, kPReady0, j & 1)) break;
         tc_fence_after();
-        issue_pv(0, j);
+        issue_pv(tmem + kTmemO, tmem + kTmemS, v_lo + stg * kTileStep, hi, j > 0);
+        mma_commit(bars + kPVDone0);
         if (more) {
-          if (!wait_bar(ctx, kKFull0 + ((j + 1) & 1), ((j + 1) >> 1) & 1)) break;
+          if (!wait_bar(ctx, kKFull0 + nstg, ((j + 1) >> 1) & 1)) break;
           tc_fence_after();
-          issue_s(0, j + 1);
+          issue_s(tmem + kTmemS, q_lo, k_lo + nstg * kTileStep, hi);
+          mma_commit(bars + kSFull0);
         }
         if (has_q1) {
           if (!wait_bar(ctx, kPReady0 + 1, j & 1)) break;
           tc_fence_after();
-          issue_pv(1, j);
-          if (more) issue_s(1, j + 1);
+          issue_pv(tmem + kTmemO + 128, tmem + kTmemS + 128, v_lo + stg * kTileStep, hi, j > 0);
+          mma_commit(bars + kPVDone0 + 1);
+          if (more) {
+            issue_s(tmem + kTmemS + 128, q_lo + kTileStep, k_lo + nstg * kTileStep, hi);
+            mma_commit(bars + kSFull0 + 1);
+          }
         }
         mma_commit(bars + kVEmpty0 + stg);
-        if (more) mma_commit(bars + kKEmpty0 + ((j + 1) & 1));
+        if (more) mma_commit(bars + kKEmpty0 + nstg);
       }
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
       mma_commit(bars + kDrain);
