@@ -42,6 +42,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="wan13b_bf16")
+    ap.add_argument("--fused", action="store_true",
+                    help="step = wf_project_publish (QKV projection + RoPE + publication from "
+                         "activations and dummy weights) + attention + advance")
     ap.add_argument("--mask", choices=["wf", "rf"], default="wf",
                     help="wf: M_WF chunk-causal mask; rf: bidirectional live window")
     ap.add_argument("--e2e-steps", type=int, default=30)
@@ -279,10 +282,23 @@ def run_ours(args, ws, rank, local):
             x[1] = torch.where(m[..., None], x[1].float() * cfg.k_outlier_scale, x[1].float()).to(tdt)
     q_rot = torch.empty(shape, dtype=tdt, device=dev)
     out = torch.empty(shape, dtype=tdt, device=dev)
+    hidden = cfg.num_heads * cfg.head_dim
+    if args.fused:
+        # activations [S+1][C][hidden] and dummy weights [3*hidden][hidden], N(0, 1/hidden)
+        acts = [torch.randn((cfg.num_slots, cfg.chunk_tokens, hidden), generator=gen, device=dev,
+                            dtype=torch.float32).to(tdt) for _ in range(2)]
+        w_qkv = (torch.randn((3 * hidden, hidden), generator=gen, device=dev, dtype=torch.float32)
+                 / math.sqrt(hidden)).to(tdt)
+
+    def publish_step(i):
+        if args.fused:
+            pool.project_publish(0, acts[i & 1], w_qkv, q_rot)
+        else:
+            x = inputs[i & 1]
+            pool.publish(0, x[0], x[1], x[2], q_rot)
 
     def step(i):
-        x = inputs[i & 1]
-        pool.publish(0, x[0], x[1], x[2], q_rot)
+        publish_step(i)
         pool.attention(0, q_rot, out)
         pool.advance()
 
@@ -311,9 +327,8 @@ def run_ours(args, ws, rank, local):
     time.sleep(0.3)
     t0.record(stream)
     for i in range(args.steps):
-        x = inputs[i & 1]
         e_pub[i][0].record(stream)
-        pool.publish(0, x[0], x[1], x[2], q_rot)
+        publish_step(i)
         e_pub[i][1].record(stream)
         e_att[i][0].record(stream)
         pool.attention(0, q_rot, out)
@@ -335,15 +350,17 @@ def run_ours(args, ws, rank, local):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
 
+    live = sum(1 for r in layout if r[2] is not None)
+    proj_flops = 2 * live * cfg.chunk_tokens * (3 * hidden) * hidden if args.fused else 0
     res = {"ms": ms, "att_ms": att_ms, "pub_ms": pub_ms, "flops": flops, "pbytes": pbytes,
-           "clocks": clk, "layout_positions": len(layout)}
+           "clocks": clk, "layout_positions": len(layout), "proj_flops": proj_flops}
 
     # End to end: the step's q, k, v come from pinned host buffers and out goes
     # back to pinned host memory, all inside the timed region. The copies are
     # pipelined the way a caller would: H2D of step i+1 on one copy stream and
     # D2H of step i-1 on another overlap the kernels of step i (double-buffered
     # device inputs and outputs, ordered by events).
-    if not args.no_e2e:
+    if not args.no_e2e and not args.fused:
         host_in = [[t.cpu().pin_memory() for t in x] for x in inputs]
         host_out = torch.empty(shape, dtype=tdt).pin_memory()
         dev_in = [[torch.empty(shape, dtype=tdt, device=dev) for _ in range(3)] for _ in range(2)]
@@ -497,12 +514,14 @@ def run_reference(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(cfg, n):
-    return {"workload": f"{cfg.name}{'' if cfg.mask == 'wf' else ' (RF mask)'}: one layer-round, S={cfg.num_stages}+store, "
+def workload_config(cfg, n, fused=False):
+    return {"workload": f"{cfg.name}{'' if cfg.mask == 'wf' else ' (RF mask)'}"
+                        f"{' (fused QKV projection)' if fused else ''}: one layer-round, S={cfg.num_stages}+store, "
                         f"C={cfg.chunk_tokens}, heads={cfg.num_heads}x{cfg.head_dim}, "
                         f"anchor={cfg.anchor_chunks}, history={cfg.history_chunks}, "
                         f"page={cfg.page_tokens}, steady state",
-            "step": "wf_publish_kv + wf_round_attention + wf_advance_round",
+            "step": ("wf_project_publish" if fused else "wf_publish_kv")
+                    + " + wf_round_attention + wf_advance_round",
             "l2": "working set > 126 MB L2 (pool 233 MB + q/k/v/q_rot/out 360 MB); no flush",
             "parallelism": f"replicas x{n}" if n > 1 else "single GPU"}
 
@@ -566,15 +585,21 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-            "config": workload_config(cfg, ws),
+            "config": workload_config(cfg, ws, args.fused),
             "rounds_per_s": ws * args.steps / (res["ms"] * 1e-3),
             "attention": {"ms_per_launch": res["att_ms"], "tflops": att_tflops,
                           "pct_bf16_peak_burst": 100 * att_tflops / peaks["bf16_tflops"],
                           "pct_bf16_peak_sustained": 100 * att_tflops / peak,
                           "flops_per_launch": res["flops"]},
-            "publish": {"ms_per_launch": res["pub_ms"], "gbs": pub_gbs,
-                        "pct_hbm": 100 * pub_gbs / peaks["hbm_gbs"],
-                        "bytes_per_launch": res["pbytes"]},
+            "publish": ({"ms_per_launch": res["pub_ms"], "gbs": pub_gbs,
+                         "pct_hbm": 100 * pub_gbs / peaks["hbm_gbs"],
+                         "bytes_per_launch": res["pbytes"]} if not args.fused else
+                        {"kernel": "project_kernel (QKV GEMM + RoPE + paged publication)",
+                         "ms_per_launch": res["pub_ms"],
+                         "gemm_tflops": res["proj_flops"] / (res["pub_ms"] * 1e-3) / 1e12,
+                         "pct_bf16_peak_burst": 100 * res["proj_flops"] / (res["pub_ms"] * 1e-3)
+                         / 1e12 / peaks["bf16_tflops"],
+                         "flops_per_launch": res["proj_flops"]}),
             "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": peak,
                          "unit": "TFLOP/s", "frac": att_tflops / peak,
                          "traffic": read_traffic(kfile),

@@ -36,6 +36,7 @@
 #include <cuda_bf16.h>
 
 #include "f32x2.cuh"
+#include "pipeline.cuh"
 #include "sm100.cuh"
 #include "wf_internal.h"
 
@@ -61,7 +62,6 @@ constexpr int kMmaWarp = 9;
 constexpr uint32_t kRegsSoftmax = 200;
 constexpr uint32_t kRegsControl = 96;
 static_assert(256 * kRegsSoftmax + 128 * kRegsControl <= 384 * 168, "register split");
-constexpr long long kWaitLimit = 2000000000LL;  // ~1 s at 2 GHz
 
 // TMEM columns.
 constexpr uint32_t kTmemS = 0;        // S_q at 128 q; P_q aliases its first 64 columns
@@ -82,43 +82,6 @@ enum Bar {
   kSFull0 = 9, kPReady0 = 11, kPVDone0 = 13, kDrain = 15
 };
 
-struct Ctx {
-  uint64_t *bars;
-  volatile int *abort;
-  int32_t *status;
-};
-
-// Bounded wait on an mbarrier phase. Returns false (and flags the CTA) on
-// timeout or when another role has already aborted.
-__device__ __forceinline__ bool wait_bar(const Ctx &c, int b, uint32_t parity) {
-  uint64_t *bar = c.bars + b;
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 127u) == 0) {
-      if (*c.abort) return false;
-      if (clock64() - t0 > kWaitLimit) {
-        *c.abort = 1;
-        record_status(c.status, WF_ERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
-// Time-bounded wait used while draining (ignores the abort flag).
-__device__ __forceinline__ void drain_wait(const Ctx &c, int b, uint32_t parity) {
-  uint64_t *bar = c.bars + b;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitLimit) {
-      record_status(c.status, WF_ERR_TIMEOUT);
-      return;
-    }
-  }
-}
-
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -134,18 +97,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);   // RNE, lo in the low half
   return *reinterpret_cast<uint32_t *>(&b);
-}
-
-// Keep the compiler from using tcgen05.ld results before tcgen05.wait::ld.
-#define WF_REG_FENCE8(r, o)                                                                 \
-  asm volatile("" : "+r"(r[o + 0]), "+r"(r[o + 1]), "+r"(r[o + 2]), "+r"(r[o + 3]),         \
-               "+r"(r[o + 4]), "+r"(r[o + 5]), "+r"(r[o + 6]), "+r"(r[o + 7]))
-
-__device__ __forceinline__ void reg_fence32(uint32_t *r) {
-  WF_REG_FENCE8(r, 0);
-  WF_REG_FENCE8(r, 8);
-  WF_REG_FENCE8(r, 16);
-  WF_REG_FENCE8(r, 24);
 }
 
 // S_q = Q_q K(stage)^T: 8 k-steps of 16 along d; Q and K are [128][128] bf16

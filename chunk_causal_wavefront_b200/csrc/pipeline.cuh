@@ -1,0 +1,68 @@
+// Bounded mbarrier waits and register fences shared by the tcgen05 kernels.
+//
+// Every wait on an mbarrier phase is bounded: after about a second of clock64
+// it records WF_ERR_TIMEOUT in the pool's status word, raises the CTA's abort
+// flag (which every other waiting role polls) and returns false, so a kernel
+// can drain its in-flight copies and MMAs, free TMEM and exit instead of
+// spinning forever.
+#pragma once
+
+#include <cstdint>
+
+#include "sm100.cuh"
+#include "wf_internal.h"
+
+namespace wf {
+
+constexpr long long kWaitLimit = 2000000000LL;  // ~1 s at 2 GHz
+
+struct Ctx {
+  uint64_t *bars;
+  volatile int *abort;
+  int32_t *status;
+};
+
+// Bounded wait on an mbarrier phase. Returns false (and flags the CTA) on
+// timeout or when another role has already aborted.
+__device__ __forceinline__ bool wait_bar(const Ctx &c, int b, uint32_t parity) {
+  uint64_t *bar = c.bars + b;
+  if (sm100::mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (sm100::mbar_try_wait(bar, parity)) return true;
+    if ((it & 127u) == 0) {
+      if (*c.abort) return false;
+      if (clock64() - t0 > kWaitLimit) {
+        *c.abort = 1;
+        record_status(c.status, WF_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Time-bounded wait used while draining (ignores the abort flag).
+__device__ __forceinline__ void drain_wait(const Ctx &c, int b, uint32_t parity) {
+  uint64_t *bar = c.bars + b;
+  const long long t0 = clock64();
+  while (!sm100::mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimit) {
+      record_status(c.status, WF_ERR_TIMEOUT);
+      return;
+    }
+  }
+}
+
+// Keep the compiler from using tcgen05.ld results before tcgen05.wait::ld.
+#define WF_REG_FENCE8(r, o)                                                                 \
+  asm volatile("" : "+r"(r[o + 0]), "+r"(r[o + 1]), "+r"(r[o + 2]), "+r"(r[o + 3]),         \
+               "+r"(r[o + 4]), "+r"(r[o + 5]), "+r"(r[o + 6]), "+r"(r[o + 7]))
+
+__device__ __forceinline__ void reg_fence32(uint32_t *r) {
+  WF_REG_FENCE8(r, 0);
+  WF_REG_FENCE8(r, 8);
+  WF_REG_FENCE8(r, 16);
+  WF_REG_FENCE8(r, 24);
+}
+
+}  // namespace wf

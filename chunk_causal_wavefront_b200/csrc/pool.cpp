@@ -451,6 +451,52 @@ wf_status wf_round_attention(wf_pool *p, int32_t layer, const void *q_rot, void 
   return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 
+wf_status wf_project_publish(wf_pool *p, int32_t layer, const void *x, const void *w_qkv,
+                             void *q_rot, wf_stream_t stream) {
+  if (!p) return WF_ERR_INVALID_ARG;
+  if (p->host_only) return WF_ERR_CALL_ORDER;
+  const wf_pool_config &c = p->cfg;
+  if (c.dtype != WF_DTYPE_BF16) return WF_ERR_UNSUPPORTED;
+  const int hidden = c.num_heads * c.head_dim;
+  if (hidden % 256 != 0 || c.page_tokens != 128) return WF_ERR_UNSUPPORTED;
+  if (layer < 0 || layer >= c.num_layers) return WF_ERR_INVALID_ARG;
+  if (!x || !w_qkv || !q_rot || !aligned16(x) || !aligned16(w_qkv) || !aligned16(q_rot))
+    return WF_ERR_INVALID_ARG;
+  if (q_rot == x || q_rot == w_qkv) return WF_ERR_INVALID_ARG;
+  if (!on_pool_device(p)) return WF_ERR_INVALID_ARG;
+  ProjectParams pp{};
+  pp.q_rot = q_rot;
+  pp.pages = p->dev + p->g.pages_off + static_cast<size_t>(layer) * p->g.num_pages * p->g.page_bytes;
+  pp.tags = reinterpret_cast<int32_t *>(p->dev + p->g.tags_off) +
+            static_cast<size_t>(layer) * p->g.num_pages;
+  pp.table = reinterpret_cast<const int32_t *>(p->dev + p->g.table_off);
+  pp.status = reinterpret_cast<int32_t *>(p->dev + p->g.status_off);
+  if (c.rope == WF_ROPE_3D) {
+    pp.rope_t = reinterpret_cast<const float2 *>(p->dev + p->g.rope_t_off);
+    pp.rope_h = reinterpret_cast<const float2 *>(p->dev + p->g.rope_h_off);
+    pp.rope_w = reinterpret_cast<const float2 *>(p->dev + p->g.rope_w_off);
+  }
+  pp.S1 = c.num_stages + 1; pp.C = c.chunk_tokens; pp.Hh = c.num_heads; pp.d = c.head_dim;
+  pp.P = c.page_tokens; pp.npc = p->g.npc; pp.num_pages = static_cast<int32_t>(p->g.num_pages);
+  pp.hidden = hidden;
+  pp.rope = c.rope; pp.F = c.frames_per_chunk; pp.gh = c.grid_h; pp.gw = c.grid_w;
+  pp.split0 = c.rope_split[0]; pp.split1 = c.rope_split[1]; pp.split2 = c.rope_split[2];
+  pp.live = live_slots(p);
+  CUtensorMap xmap, wmap;
+  const cuuint64_t xd[3] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(c.chunk_tokens),
+                            static_cast<cuuint64_t>(c.num_stages + 1)};
+  const cuuint64_t xs[2] = {static_cast<cuuint64_t>(hidden) * 2,
+                            static_cast<cuuint64_t>(hidden) * 2 * c.chunk_tokens};
+  const cuuint32_t xb[3] = {64, 128, 1};
+  if (!encode_bf16_map(&xmap, const_cast<void *>(x), 3, xd, xs, xb)) return WF_ERR_CUDA;
+  const cuuint64_t wd[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(3 * hidden)};
+  const cuuint64_t ws[1] = {static_cast<cuuint64_t>(hidden) * 2};
+  const cuuint32_t wb[2] = {64, 256};
+  if (!encode_bf16_map(&wmap, const_cast<void *>(w_qkv), 2, wd, ws, wb)) return WF_ERR_CUDA;
+  cudaError_t e = launch_project_bf16(pp, &xmap, &wmap, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
 wf_status wf_advance_round(wf_pool *p, wf_stream_t stream) {
   if (!p) return WF_ERR_INVALID_ARG;
   const int S = p->cfg.num_stages;

@@ -1,0 +1,241 @@
+// Fused QKV projection + 3D rotary + early publication, tcgen05 GEMM for sm_100a.
+//
+// "Wave Forcing: Towards Speed-of-Light Streaming Video Generation", Method
+// section: each rank's local QKV projection runs without waiting for remote
+// K/V, and K/V are published right after the QKV projection and RoPE, with
+// direct writes into ordered attention slots. Here the projection's epilogue
+// is the publication: q_rot is written, K and V go straight into the slot's
+// pages, the rows past C in the chunk's last page are zeroed and the ready tag
+// is stamped, so q, k and v never make a round trip through HBM.
+//
+// Y[token][f] = sum_i x[token][i] * w[f][i] for the live slots' tokens, with
+// f over the 3 * hidden stacked q, k, v output features.
+//   CTA tile: 128 tokens (exactly one 128-token page of the slot's chunk) x
+//   256 output features (two heads of q, k or v); hidden is walked in
+//   64-element (128-byte) blocks through a 4-stage TMA ring (128-byte swizzle,
+//   A = x tile, B = w tile, both K-major).
+//   warp 4 (one lane)  TMA producer;
+//   warp 5 (one lane)  tcgen05 issuer: M = 128, N = 256, K = 16, fp32
+//                      accumulation in 256 TMEM columns;
+//   warps 0-3          epilogue: thread r owns token r (TMEM lane r), loads its
+//                      row 32 columns at a time, rotates q and k pairs in fp32
+//                      with the pool's (cos, sin) tables, rounds once to bf16
+//                      and stores 64-byte pieces to q_rot or to the page row.
+// Order of CTAs: feature tiles fastest, so consecutive CTAs share the x tile
+// and sweep w (14 MB for the 1.3B shape), which both stay in L2.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "pipeline.cuh"
+#include "sm100.cuh"
+#include "wf_internal.h"
+
+namespace wf {
+namespace {
+
+using namespace sm100;
+
+constexpr int kGM = 128;                      // tokens per tile
+constexpr int kGN = 256;                      // output features per tile
+constexpr int kGK = 64;                       // hidden elements per k-block
+constexpr int kStages = 4;
+constexpr uint32_t kABytes = kGM * kGK * 2;   // 16 KB
+constexpr uint32_t kBBytes = kGN * kGK * 2;   // 32 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr uint32_t kOffBar = kStages * kStageBytes;
+enum { kFull0 = 0, kEmpty0 = kStages, kAccFull = 2 * kStages, kDrain = 2 * kStages + 1,
+       kNumBars = 2 * kStages + 2 };
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;   // + alignment slack
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&b);
+}
+
+// Rotate the 16 pairs of a 32-column piece whose first column is dimension
+// dim0 of its head, for a token at rotary position (t, y, x).
+__device__ __forceinline__ void rope32(float *v, int dim0, int t, int y, int x,
+                                       const ProjectParams &p) {
+  const int h0 = p.split0 >> 1, h1 = p.split1 >> 1, h2 = p.split2 >> 1;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int pr = (dim0 >> 1) + i;
+    float2 cs;
+    if (pr < h0) cs = __ldg(p.rope_t + t * h0 + pr);
+    else if (pr < h0 + h1) cs = __ldg(p.rope_h + y * h1 + (pr - h0));
+    else cs = __ldg(p.rope_w + x * h2 + (pr - h0 - h1));
+    const float a = v[2 * i], b = v[2 * i + 1];
+    v[2 * i] = a * cs.x - b * cs.y;
+    v[2 * i + 1] = a * cs.y + b * cs.x;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    project_kernel(const __grid_constant__ ProjectParams p, const __grid_constant__ CUtensorMap tx,
+                   const __grid_constant__ CUtensorMap tw) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int n_tiles = 3 * p.hidden / kGN;
+  const int nt = blockIdx.x % n_tiles;
+  const int rest = blockIdx.x / n_tiles;
+  const int mt = rest % p.npc;                  // token tile == page of the chunk
+  const int li = rest / p.npc;
+  const int slot = p.live.slot[li];
+  const int n_kb = p.hidden / kGK;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int b = 0; b < kNumBars; ++b) mbar_init(bars + b, 1);
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Ctx ctx{bars, abort_flag, p.status};
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tx);
+      tma_prefetch_desc(&tw);
+      int issued = 0;
+      for (int kb = 0; kb < n_kb; ++kb) {
+        const int s = kb % kStages;
+        if (!wait_bar(ctx, kEmpty0 + s, ((kb / kStages) & 1) ^ 1)) break;
+        uint8_t *sa = smem + s * kStageBytes;
+        mbar_arrive_expect_tx(bars + kFull0 + s, kStageBytes);
+        tma_load_3d(sa, &tx, bars + kFull0 + s, kb * kGK, mt * kGM, slot);
+        tma_load_2d(sa + kABytes, &tw, bars + kFull0 + s, kb * kGK, nt * kGN);
+        issued = kb + 1;
+      }
+      // Drain: the last load of every stage has landed before the CTA exits.
+      for (int kb = issued - kStages < 0 ? 0 : issued - kStages; kb < issued; ++kb)
+        drain_wait(ctx, kFull0 + kb % kStages, (kb / kStages) & 1);
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc_bf16(kGM, kGN, false);
+      const uint32_t hi = desc_hi_sw128(1024);
+      const uint32_t lo0 = desc_lo_sw128(smem_u32(smem), 16);
+      bool ok = true;
+      for (int kb = 0; kb < n_kb; ++kb) {
+        const int s = kb % kStages;
+        if (!wait_bar(ctx, kFull0 + s, (kb / kStages) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_lo = lo0 + ((s * kStageBytes) >> 4);
+        const uint32_t b_lo = a_lo + (kABytes >> 4);
+#pragma unroll
+        for (int k = 0; k < kGK / 16; ++k)
+          mma_bf16_ss2(tmem, a_lo + k * 2, b_lo + k * 2, hi, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+        mma_commit(bars + kEmpty0 + s);
+      }
+      if (ok) mma_commit(bars + kAccFull);
+      mma_commit(bars + kDrain);
+      drain_wait(ctx, kDrain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue --
+    const int r = warp * 32 + lane;                      // token row == TMEM lane
+    const int n = mt * kGM + r;                          // token inside the chunk
+    const bool valid = n < p.C;
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const bool ok = __all_sync(0xffffffffu, wait_bar(ctx, kAccFull, 0));
+    if (ok) {
+      tc_fence_after();
+      int tpos = 0, ypos = 0, xpos = 0;
+      if (p.rope && valid) {
+        const int hw = p.gh * p.gw;
+        tpos = p.F * p.live.chunk[li] + n / hw;
+        ypos = (n / p.gw) % p.gh;
+        xpos = n % p.gw;
+      }
+      const int pos = __ldg(p.table + kTabSlotPos + slot);
+      int phys = pos < 0 ? -1 : __ldg(p.table + kTabPages + pos * p.npc + mt);
+      if (phys >= p.num_pages) phys = -1;
+      const size_t page_elems = static_cast<size_t>(2) * p.Hh * p.P * p.d;
+#pragma unroll 1
+      for (int c = 0; c < kGN / 32; ++c) {
+        uint32_t raw[32];
+        tmem_ld32(tmem + lane_addr + c * 32, raw);
+        tmem_ld_wait();
+        reg_fence32(raw);
+        const int f0 = nt * kGN + c * 32;                // first output feature of the piece
+        const int sec = f0 / p.hidden;                   // 0 q, 1 k, 2 v
+        const int within = f0 - sec * p.hidden;
+        const int head = within / p.d;
+        const int dim0 = within - head * p.d;
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+        if (sec < 2 && p.rope && valid) rope32(v, dim0, tpos, ypos, xpos, p);
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = valid ? pack_bf16(v[2 * i], v[2 * i + 1]) : 0u;
+        // Lanes decide independently whether and where to store; the warp
+        // stays converged for the next tcgen05.ld.
+        uint4 *dst = nullptr;
+        if (sec == 0) {
+          if (valid)
+            dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.q_rot) +
+                                            ((static_cast<size_t>(slot) * p.C + n) * p.Hh + head) *
+                                                p.d + dim0);
+        } else if (phys < 0) {
+          record_status(p.status, WF_ERR_BAD_PAGE);
+        } else {
+          dst = reinterpret_cast<uint4 *>(
+              reinterpret_cast<__nv_bfloat16 *>(p.pages) + phys * page_elems +
+              ((static_cast<size_t>(sec - 1) * p.Hh + head) * p.P + r) * p.d + dim0);
+          if (sec == 1 && head == 0 && dim0 == 0 && r == 0) p.tags[phys] = p.live.tag[li];
+        }
+        if (dst != nullptr) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+        __syncwarp();
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_project_bf16(const ProjectParams &p, const void *tmap_x, const void *tmap_w,
+                                cudaStream_t st) {
+  if (p.live.n == 0) return cudaSuccess;
+  if (p.d != 128 || p.P != kGM || p.hidden % kGN != 0) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = static_cast<int64_t>(p.live.n) * p.npc * (3 * p.hidden / kGN);
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  project_kernel<<<static_cast<unsigned>(blocks), kThreads, kSmemBytes, st>>>(
+      p, *static_cast<const CUtensorMap *>(tmap_x), *static_cast<const CUtensorMap *>(tmap_w));
+  return cudaGetLastError();
+}
+
+}  // namespace wf

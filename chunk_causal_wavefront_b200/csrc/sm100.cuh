@@ -63,6 +63,15 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *desc, uint64_
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_3d(void *dst, const void *desc, uint64_t *bar, int x,
+                                            int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(desc), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_4d(void *dst, const void *desc, uint64_t *bar, int x,
                                             int y, int z, int w) {
   asm volatile(

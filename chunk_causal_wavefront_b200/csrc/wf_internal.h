@@ -65,6 +65,18 @@ struct AttnParams {
   LiveSlots live;
 };
 
+struct ProjectParams {
+  void *q_rot;
+  char *pages;                // this layer's page region
+  int32_t *tags;              // this layer's ready tags
+  const int32_t *table;
+  int32_t *status;
+  const float2 *rope_t, *rope_h, *rope_w;
+  int32_t S1, C, Hh, d, P, npc, num_pages, hidden;
+  int32_t rope, F, gh, gw, split0, split1, split2;
+  LiveSlots live;
+};
+
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_publish_bf16(const PublishParams &p, cudaStream_t st);
 cudaError_t launch_publish_f32(const PublishParams &p, cudaStream_t st);
@@ -75,6 +87,10 @@ cudaError_t launch_attention_f32(const AttnParams &p, cudaStream_t st);
 cudaError_t launch_attention_bf16(const AttnParams &p, const void *tmap_q,
                                   const void *tmap_kv, const void *tmap_out,
                                   cudaStream_t st);
+// Fused QKV projection: tensor maps of x (3D: hidden x C x S+1, box 64 x 128 x 1)
+// and w_qkv (2D: hidden x 3*hidden, box 64 x 256).
+cudaError_t launch_project_bf16(const ProjectParams &p, const void *tmap_x, const void *tmap_w,
+                                cudaStream_t st);
 cudaError_t launch_table_upload(int32_t *dst, const int32_t *src, int n_words,
                                 cudaStream_t st);
 cudaError_t launch_poke(int32_t *dst, int32_t value, cudaStream_t st);

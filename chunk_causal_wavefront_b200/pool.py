@@ -84,6 +84,13 @@ class KVPool:
         if st != _wf.WF_OK:
             raise WfError(st, "wf_publish_kv")
 
+    def project_publish(self, layer: int, x: torch.Tensor, w_qkv: torch.Tensor,
+                        q_rot: torch.Tensor, stream=None) -> None:
+        st = _wf.wf_project_publish(self.handle, layer, _ptr(x), _ptr(w_qkv), _ptr(q_rot),
+                                    _stream(self.device, stream))
+        if st != _wf.WF_OK:
+            raise WfError(st, "wf_project_publish")
+
     def attention(self, layer: int, q_rot: torch.Tensor, out: torch.Tensor, stream=None) -> None:
         st = _wf.wf_round_attention(self.handle, layer, _ptr(q_rot), _ptr(out),
                                     _stream(self.device, stream))

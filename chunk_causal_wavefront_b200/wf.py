@@ -34,6 +34,7 @@ EXPORTS = (
     "wf_kv_pool_bytes", "wf_kv_pool_create", "wf_publish_kv", "wf_round_attention",
     "wf_advance_round", "wf_pool_check_status", "wf_pool_destroy", "wf_status_string",
     "wf_pool_round", "wf_pool_get_geometry", "wf_pool_get_layout", "wf_pool_debug_poke_page",
+    "wf_project_publish",
 )
 
 
@@ -89,6 +90,7 @@ def _load():
         "wf_pool_get_geometry": (I32, [P, ctypes.POINTER(WfPoolGeometry)]),
         "wf_pool_get_layout": (I32, [P, i32p, i32p, i32p, i32p, i32p, i32p, I32]),
         "wf_pool_debug_poke_page": (I32, [P, I32, I32, I32, P]),
+        "wf_project_publish": (I32, [P, I32, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -185,3 +187,7 @@ def wf_pool_debug_poke_page(pool: int, position: int, j: int, physical: int, str
     return _lib.wf_pool_debug_poke_page(pool, position, j, physical,
                                         ctypes.c_void_p(stream or None))
 
+
+
+def wf_project_publish(pool: int, layer: int, x: int, w_qkv: int, q_rot: int, stream: int) -> int:
+    return _lib.wf_project_publish(pool, layer, x, w_qkv, q_rot, ctypes.c_void_p(stream or None))

@@ -154,6 +154,24 @@ wf_status wf_publish_kv(wf_pool *pool, int32_t layer, const void *q, const void 
 wf_status wf_round_attention(wf_pool *pool, int32_t layer, const void *q_rot, void *out,
                              wf_stream_t stream);
 
+/* Fused QKV projection + publication for one layer (Method section: the local
+ * QKV projection runs without waiting for remote K/V, and K/V are published
+ * right after the projection and RoPE, written straight into the ordered
+ * slots). For every live slot s and token n:
+ *     [q | k | v][s][n] = x[s][n] . w_qkv^T        (fp32 accumulation)
+ * then q and k are rotated by the 3D rotary embedding exactly as in
+ * wf_publish_kv, and the results are written as wf_publish_kv writes them:
+ * q_rot rows, K and V page rows (rows past C zeroed), ready tags.
+ *   x     : [S+1][C][hidden] bf16 activations, hidden = num_heads * head_dim;
+ *           rows of slots that are not live are not read.
+ *   w_qkv : [3 * hidden][hidden] bf16, the q, k, v output features stacked
+ *           (row f holds the weights of output feature f).
+ *   q_rot : [S+1][C][heads][d] bf16; only live slots' rows are written.
+ * bf16 pools only, with head_dim 128, page_tokens 128 and hidden a multiple of
+ * 256 (WF_ERR_UNSUPPORTED otherwise). Pointers must be 16-byte aligned. */
+wf_status wf_project_publish(wf_pool *pool, int32_t layer, const void *x, const void *w_qkv,
+                             void *q_rot, wf_stream_t stream);
+
 /* Move the pool to the next round (k -> k + 1, Table 3): the store's chunk
  * becomes the anchor (chunk 0, when kept) or the newest history chunk; history
  * beyond H returns its pages to the free list; the next store takes pages

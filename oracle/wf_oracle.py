@@ -54,6 +54,7 @@ __all__ = [
     "Position", "round_layout", "visible_positions", "rope_positions", "rope_3d",
     "attention_slot_prefix", "attention_dense_mask", "attention_bruteforce",
     "PoolModel", "expected_tag", "publish_pages", "unmasked_flops", "round_bf16",
+    "project_qkv",
 ]
 
 
@@ -158,6 +159,25 @@ def rope_3d(x: np.ndarray, chunk: int, F: int, gh: int, gw: int,
         out[:, :, off + 1:off + da:2] = a * s + b * c
         off += da
     return out
+
+
+# ---------------------------------------------------------------------------
+# QKV projection (the local step before publication).
+# ---------------------------------------------------------------------------
+
+def project_qkv(x: np.ndarray, w_qkv: np.ndarray, heads: int, d: int):
+    """q, k, v = x W_q^T, x W_k^T, x W_v^T for one chunk, in float64.
+
+    x: [C][hidden] activations; w_qkv: [3 * hidden][hidden] with the q, k and v
+    output features stacked (the per-rank QKV projection that runs before
+    RoPE and publication, Method section). Returns three [C][heads][d] arrays.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w_qkv, dtype=np.float64)
+    hidden = heads * d
+    y = x @ w.T                                   # library matmul as one step
+    return tuple(y[:, i * hidden:(i + 1) * hidden].reshape(x.shape[0], heads, d)
+                 for i in range(3))
 
 
 # ---------------------------------------------------------------------------

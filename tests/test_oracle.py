@@ -365,3 +365,21 @@ def test_rf_work_closed_form():
     S, A, H = 4, 1, 2
     k = S + A + H + 1
     assert O.unmasked_flops(S, A, H, k, 7, 2, 8, "rf") == 4 * 7 * 7 * 8 * 2 * (S + 1) * (A + H + S + 1)
+
+
+# --- QKV projection -----------------------------------------------------------
+
+def test_project_qkv_against_elementwise_sums():
+    rng = np.random.default_rng(11)
+    C, heads, d = 5, 2, 4
+    hidden = heads * d
+    x = rng.standard_normal((C, hidden))
+    w = rng.standard_normal((3 * hidden, hidden))
+    q, k, v = O.project_qkv(x, w, heads, d)
+    for which, out in enumerate((q, k, v)):
+        for n in range(C):
+            for h in range(heads):
+                for c in range(d):
+                    f = which * hidden + h * d + c        # output feature index
+                    want = sum(x[n, i] * w[f, i] for i in range(hidden))
+                    assert out[n, h, c] == pytest.approx(want, abs=1e-12)
