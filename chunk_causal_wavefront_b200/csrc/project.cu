@@ -10,17 +10,21 @@
 //
 // Y[token][f] = sum_i x[token][i] * w[f][i] for the live slots' tokens, with
 // f over the 3 * hidden stacked q, k, v output features.
-//   CTA tile: 128 tokens (exactly one 128-token page of the slot's chunk) x
+//   CTA tile: 256 tokens (exactly two 128-token pages of the slot's chunk) x
 //   256 output features (two heads of q, k or v); hidden is walked in
-//   64-element (128-byte) blocks through a 4-stage TMA ring (128-byte swizzle,
-//   A = x tile, B = w tile, both K-major).
-//   warp 4 (one lane)  TMA producer;
-//   warp 5 (one lane)  tcgen05 issuer: M = 128, N = 256, K = 16, fp32
-//                      accumulation in 256 TMEM columns;
-//   warps 0-3          epilogue: thread r owns token r (TMEM lane r), loads its
-//                      row 32 columns at a time, rotates q and k pairs in fp32
-//                      with the pool's (cos, sin) tables, rounds once to bf16
-//                      and stores 64-byte pieces to q_rot or to the page row.
+//   64-element (128-byte) blocks through a 3-stage TMA ring (128-byte swizzle,
+//   A = x tile, B = w tile, both K-major). Each 256 x 256 tile reads 128 FLOP
+//   per byte of operands (a 128-token tile would read 85), which matters
+//   because the operands come from L2.
+//   warp 8 (one lane)  TMA producer;
+//   warp 9 (one lane)  tcgen05 issuer: two M = 128, N = 256, K = 16 MMAs per
+//                      k-step (one per page of the tile), fp32 accumulation
+//                      in TMEM columns [0, 256) and [256, 512);
+//   warps 0-7          epilogue, one warpgroup per page: thread r owns token r
+//                      of its page (TMEM lane r), loads its row 32 columns at a
+//                      time, rotates q and k pairs in fp32 with the pool's
+//                      (cos, sin) tables, rounds once to bf16 and stores
+//                      64-byte pieces to q_rot or to the page row.
 // Order of CTAs: feature tiles fastest, so consecutive CTAs share the x tile
 // and sweep w (14 MB for the 1.3B shape), which both stay in L2.
 #include <cuda.h>
@@ -35,16 +39,17 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kGM = 128;                      // tokens per tile
+constexpr int kPage = 128;                    // tokens per page (and per MMA, M)
+constexpr int kGM = 2 * kPage;                // tokens per tile
 constexpr int kGN = 256;                      // output features per tile
 constexpr int kGK = 64;                       // hidden elements per k-block
-constexpr int kStages = 4;
-constexpr uint32_t kABytes = kGM * kGK * 2;   // 16 KB
+constexpr int kStages = 3;
+constexpr uint32_t kABytes = kGM * kGK * 2;   // 32 KB
 constexpr uint32_t kBBytes = kGN * kGK * 2;   // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr uint32_t kOffBar = kStages * kStageBytes;
 enum { kFull0 = 0, kEmpty0 = kStages, kAccFull = 2 * kStages, kDrain = 2 * kStages + 1,
        kNumBars = 2 * kStages + 2 };
@@ -86,10 +91,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int n_tiles = 3 * p.hidden / kGN;
+  const int m_tiles = (p.npc + 1) / 2;
   const int nt = blockIdx.x % n_tiles;
   const int rest = blockIdx.x / n_tiles;
-  const int mt = rest % p.npc;                  // token tile == page of the chunk
-  const int li = rest / p.npc;
+  const int mt = rest % m_tiles;                // token tile == pages 2 mt, 2 mt + 1
+  const int li = rest / m_tiles;
   const int slot = p.live.slot[li];
   const int n_kb = p.hidden / kGK;
 
@@ -99,7 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -128,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc_bf16(kGM, kGN, false);
+      constexpr uint32_t idesc = make_idesc_bf16(kPage, kGN, false);
       const uint32_t hi = desc_hi_sw128(1024);
       const uint32_t lo0 = desc_lo_sw128(smem_u32(smem), 16);
       bool ok = true;
@@ -142,8 +148,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_lo = lo0 + ((s * kStageBytes) >> 4);
         const uint32_t b_lo = a_lo + (kABytes >> 4);
 #pragma unroll
-        for (int k = 0; k < kGK / 16; ++k)
-          mma_bf16_ss2(tmem, a_lo + k * 2, b_lo + k * 2, hi, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+        for (int k = 0; k < kGK / 16; ++k) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h)   // rows 128 h .. 128 h + 127 of the A tile
+            mma_bf16_ss2(tmem + h * kGN, a_lo + ((h * kPage * 128) >> 4) + k * 2, b_lo + k * 2,
+                         hi, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+        }
         mma_commit(bars + kEmpty0 + s);
       }
       if (ok) mma_commit(bars + kAccFull);
@@ -152,12 +162,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue --
-    const int r = warp * 32 + lane;                      // token row == TMEM lane
-    const int n = mt * kGM + r;                          // token inside the chunk
+    const int h = warp >> 2;                             // page of the tile
+    const int page = 2 * mt + h;                         // page of the chunk
+    const int r = (warp & 3) * 32 + lane;                // token row in the page == TMEM lane
+    const int n = page * kPage + r;                      // token inside the chunk
     const bool valid = n < p.C;
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const bool ok = __all_sync(0xffffffffu, wait_bar(ctx, kAccFull, 0));
-    if (ok) {
+    if (ok && page < p.npc) {
       tc_fence_after();
       int tpos = 0, ypos = 0, xpos = 0;
       if (p.rope && valid) {
@@ -167,13 +179,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         xpos = n % p.gw;
       }
       const int pos = __ldg(p.table + kTabSlotPos + slot);
-      int phys = pos < 0 ? -1 : __ldg(p.table + kTabPages + pos * p.npc + mt);
+      int phys = pos < 0 ? -1 : __ldg(p.table + kTabPages + pos * p.npc + page);
       if (phys >= p.num_pages) phys = -1;
       const size_t page_elems = static_cast<size_t>(2) * p.Hh * p.P * p.d;
 #pragma unroll 1
       for (int c = 0; c < kGN / 32; ++c) {
         uint32_t raw[32];
-        tmem_ld32(tmem + lane_addr + c * 32, raw);
+        tmem_ld32(tmem + lane_addr + h * kGN + c * 32, raw);
         tmem_ld_wait();
         reg_fence32(raw);
         const int f0 = nt * kGN + c * 32;                // first output feature of the piece
@@ -218,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -227,11 +239,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 cudaError_t launch_project_bf16(const ProjectParams &p, const void *tmap_x, const void *tmap_w,
                                 cudaStream_t st) {
   if (p.live.n == 0) return cudaSuccess;
-  if (p.d != 128 || p.P != kGM || p.hidden % kGN != 0) return cudaErrorInvalidValue;
+  if (p.d != 128 || p.P != kPage || p.hidden % kGN != 0) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  const int64_t blocks = static_cast<int64_t>(p.live.n) * p.npc * (3 * p.hidden / kGN);
+  const int64_t blocks = static_cast<int64_t>(p.live.n) * ((p.npc + 1) / 2) * (3 * p.hidden / kGN);
   if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
   project_kernel<<<static_cast<unsigned>(blocks), kThreads, kSmemBytes, st>>>(
       p, *static_cast<const CUtensorMap *>(tmap_x), *static_cast<const CUtensorMap *>(tmap_w));

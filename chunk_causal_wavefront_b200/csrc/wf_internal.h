@@ -87,7 +87,7 @@ cudaError_t launch_attention_f32(const AttnParams &p, cudaStream_t st);
 cudaError_t launch_attention_bf16(const AttnParams &p, const void *tmap_q,
                                   const void *tmap_kv, const void *tmap_out,
                                   cudaStream_t st);
-// Fused QKV projection: tensor maps of x (3D: hidden x C x S+1, box 64 x 128 x 1)
+// Fused QKV projection: tensor maps of x (3D: hidden x C x S+1, box 64 x 256 x 1)
 // and w_qkv (2D: hidden x 3*hidden, box 64 x 256).
 cudaError_t launch_project_bf16(const ProjectParams &p, const void *tmap_x, const void *tmap_w,
                                 cudaStream_t st);
