@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=None,
+                    help="oracle time per reference step (default: ~150 s over the run)")
     return ap.parse_args()
 
 
@@ -61,6 +63,28 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return ws, rank, local
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity when not
+    distributed). Uses a tensor on ``device`` (the rank's GPU under NCCL, the
+    CPU under gloo)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    if device is None:
+        device = torch.device("cpu") if dist.get_backend() == "gloo" else torch.device(
+            "cuda", torch.cuda.current_device())
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_rate(units_per_rank, ms_max, n_ranks):
+    """Units per second of the whole job: every rank processes units_per_rank
+    in its timed region, and the job takes as long as its slowest rank."""
+    return n_ranks * units_per_rank / (ms_max * 1e-3)
 
 
 def read_peaks():
@@ -237,10 +261,7 @@ def run_stream(args, ws, rank, local):
     steady = cfg.steady_round()
     ms = sum(per)
     steady_ms = sum(per[steady:]) if rounds > steady else float("nan")
-    if ws > 1:
-        t = torch.tensor([ms, steady_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, steady_ms = (float(x) for x in t.tolist())
+    ms, steady_ms = max_over_ranks([ms, steady_ms], dev)
     pool.close()
     return {"ms": ms, "steady_ms": steady_ms, "flops_total": sum(flops),
             "flops_steady": sum(flops[steady:]), "rounds": rounds, "steady_rounds": max(0, rounds - steady),
@@ -345,10 +366,7 @@ def run_ours(args, ws, rank, local):
     ms = t0.elapsed_time(t1)
     att_ms = statistics.mean(a.elapsed_time(b) for a, b in e_att)
     pub_ms = statistics.mean(a.elapsed_time(b) for a, b in e_pub)
-    if ws > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms, = max_over_ranks([ms], dev)
 
     live = sum(1 for r in layout if r[2] is not None)
     proj_flops = 2 * live * cfg.chunk_tokens * (3 * hidden) * hidden if args.fused else 0
@@ -411,10 +429,7 @@ def run_ours(args, ws, rank, local):
         b.record(stream)
         torch.cuda.synchronize()
         e_ms = a.elapsed_time(b)
-        if ws > 1:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms, = max_over_ranks([e_ms], dev)
         res["e2e"] = {"ms": e_ms, "steps": args.e2e_steps, "h2d": h2d, "d2h": d2h}
         st = pool.check_status()
         if st != 0:
@@ -492,7 +507,8 @@ def run_reference(args, ws, rank):
     cfg = wf_inputs.CONFIGS[args.config]
     if rank != 0:
         return
-    per_step = max(0.5, min(4.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step = (args.ref_step_seconds if args.ref_step_seconds is not None
+                else max(0.5, min(4.0, 150.0 / max(1, args.steps + args.warmup))))
     for _ in range(args.warmup):
         oracle_sample_rate(cfg, per_step / 4)
     rates = []
@@ -546,7 +562,7 @@ def main():
     if cfg.num_layers > 1:
         res = run_stream(args, ws, rank, local)
         if rank == 0:
-            value = ws * res["flops_total"] / (res["ms"] * 1e-3) / 1e12
+            value = whole_job_rate(res["flops_total"], res["ms"], ws) / 1e12
             line = {
                 "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": res["rounds"],
                 "warmup": args.warmup, "ms_per_step": res["ms"] / res["rounds"],
@@ -576,7 +592,7 @@ def main():
     if rank == 0:
         peaks, src = read_peaks()
         ms_step = res["ms"] / args.steps
-        value = ws * res["flops"] * args.steps / (res["ms"] * 1e-3) / 1e12
+        value = whole_job_rate(res["flops"] * args.steps, res["ms"], ws) / 1e12
         att_tflops = res["flops"] / (res["att_ms"] * 1e-3) / 1e12
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         pub_gbs = res["pbytes"] / (res["pub_ms"] * 1e-3) / 1e9
