@@ -25,8 +25,8 @@ Readings taken here (each listed in the design notes of the repository):
     block's largest magnitude lands in [224, 448];
   * Q and K are rotated (3D rotary) in float32 before quantisation: each
     product and each sum rounded once to float32 (no fused multiply-add), with
-    the (cos, sin) tables computed in float64 and rounded to float32. V is
-    quantised from its bf16 value;
+    the (cos, sin) tables computed in float64 by the C library's pow, cos and
+    sin and rounded to float32. V is quantised from its bf16 value;
   * rows of a chunk's last page past C are zero codes; query tiles cover rows
     [128 t, 128 t + 128) clipped at C.
 
@@ -112,11 +112,22 @@ def quantize_block(x32: np.ndarray):
 
 
 def rope_tables_f32(n_pos: int, width: int, base: float):
-    """(cos, sin) [n_pos][width/2] of pos * base^(-2m/width), float64 rounded to float32."""
-    m = np.arange(width // 2, dtype=np.float64)
-    inv = np.power(float(base), -2.0 * m / float(width))
-    ang = np.arange(n_pos, dtype=np.float64)[:, None] * inv[None, :]
-    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+    """(cos, sin) [n_pos][width/2] of pos * base^(-2m/width), float64 rounded to float32.
+
+    The float64 values come from the C library's pow, cos and sin (Python's
+    math module), the double-precision routines a host program calls: NumPy's
+    vectorised pow may differ from them in the last bit, which can move a
+    float32-rounded table entry and, through it, an E4M3 code."""
+    half = width // 2
+    cos_t = np.empty((n_pos, half), dtype=np.float32)
+    sin_t = np.empty((n_pos, half), dtype=np.float32)
+    for m in range(half):
+        inv = math.pow(float(base), -2.0 * m / float(width))
+        for pos in range(n_pos):
+            ang = float(pos) * inv
+            cos_t[pos, m] = math.cos(ang)
+            sin_t[pos, m] = math.sin(ang)
+    return cos_t, sin_t
 
 
 def rope_3d_f32(x32: np.ndarray, chunk: int, F: int, gh: int, gw: int,
