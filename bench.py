@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--fused", action="store_true",
                     help="step = wf_project_publish (QKV projection + RoPE + publication from "
                          "activations and dummy weights) + attention + advance")
+    ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16",
+                    help="pool storage: bf16, or E4M3 codes with block scales and FP8 "
+                         "tensor-core attention")
     ap.add_argument("--mask", choices=["wf", "rf"], default="wf",
                     help="wf: M_WF chunk-causal mask; rf: bidirectional live window")
     ap.add_argument("--e2e-steps", type=int, default=30)
@@ -101,7 +104,7 @@ def source_sha(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def read_traffic(kernel_file):
+def read_traffic(kernel_file, variant=None):
     """Per-launch DRAM bytes of a kernel from the committed ncu summary, or None
     when the kernel source has changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
@@ -109,7 +112,8 @@ def read_traffic(kernel_file):
         return None
     with open(p) as f:
         d = json.load(f)
-    e = d.get(os.path.basename(kernel_file))
+    key = os.path.basename(kernel_file) + (f":{variant}" if variant else "")
+    e = d.get(key)
     if not e or e.get("source_sha") != source_sha(kernel_file):
         return None
     return e.get("dram_bytes_per_launch")
@@ -179,14 +183,17 @@ def unmasked_flops(layout, cfg):
     return total
 
 
-def publish_bytes(layout, cfg):
+def publish_bytes(layout, cfg, kv="bf16"):
     """Algorithmic HBM bytes of one publish: read q, k, v and write q_rot, K, V
-    pages (rows of live slots; the zeroed page tail counted as written)."""
+    pages (rows of live slots; the zeroed page tail counted as written). FP8
+    pools read bf16 and write 1-byte codes plus one fp32 scale per block."""
     live = sum(1 for r in layout if r[2] is not None)
-    elt = 2 if cfg.dtype == "bf16" else 4
-    row = cfg.num_heads * cfg.head_dim * elt
+    elt_in = 2 if cfg.dtype == "bf16" else 4
+    elt_out = 1 if kv == "fp8" else elt_in
+    hd = cfg.num_heads * cfg.head_dim
     tail = cfg.pages_per_chunk * cfg.page_tokens - cfg.chunk_tokens
-    return live * (6 * cfg.chunk_tokens * row + 2 * tail * row)
+    scales = 3 * cfg.pages_per_chunk * cfg.num_heads * 4 if kv == "fp8" else 0
+    return live * (3 * cfg.chunk_tokens * hd * (elt_in + elt_out) + 2 * tail * hd * elt_out + scales)
 
 
 # ------------------------------------------------------------------------- our arm
@@ -284,7 +291,8 @@ def run_ours(args, ws, rank, local):
     pool = KVPool(make_config(num_stages=cfg.num_stages, chunk_tokens=cfg.chunk_tokens,
                               num_heads=cfg.num_heads, head_dim=cfg.head_dim,
                               anchor_chunks=cfg.anchor_chunks, history_chunks=cfg.history_chunks,
-                              page_tokens=cfg.page_tokens, num_layers=1, dtype=cfg.dtype,
+                              page_tokens=cfg.page_tokens, num_layers=1,
+                              dtype="fp8" if args.kv == "fp8" else cfg.dtype,
                               rope=cfg.rope, frames_per_chunk=cfg.frames_per_chunk,
                               grid_h=cfg.grid_h, grid_w=cfg.grid_w, rope_split=cfg.rope_split,
                               rope_base=cfg.rope_base, max_rounds=total_rounds, mask=cfg.mask),
@@ -301,7 +309,7 @@ def run_ours(args, ws, rank, local):
         for x in inputs:
             m = torch.rand(shape[:3], generator=gen, device=dev) < cfg.k_outlier_frac
             x[1] = torch.where(m[..., None], x[1].float() * cfg.k_outlier_scale, x[1].float()).to(tdt)
-    q_rot = torch.empty(shape, dtype=tdt, device=dev)
+    q_rot = torch.empty(shape, dtype=torch.uint8 if args.kv == "fp8" else tdt, device=dev)
     out = torch.empty(shape, dtype=tdt, device=dev)
     hidden = cfg.num_heads * cfg.head_dim
     if args.fused:
@@ -333,7 +341,7 @@ def run_ours(args, ws, rank, local):
         raise RuntimeError(f"device status {st} after warm-up")
     layout = pool.layout()
     flops = unmasked_flops(layout, cfg)
-    pbytes = publish_bytes(layout, cfg)
+    pbytes = publish_bytes(layout, cfg, args.kv)
 
     import torch.distributed as dist
     ev = lambda: torch.cuda.Event(enable_timing=True)
@@ -530,9 +538,11 @@ def run_reference(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(cfg, n, fused=False):
+def workload_config(cfg, n, fused=False, kv="bf16"):
     return {"workload": f"{cfg.name}{'' if cfg.mask == 'wf' else ' (RF mask)'}"
-                        f"{' (fused QKV projection)' if fused else ''}: one layer-round, S={cfg.num_stages}+store, "
+                        f"{' (fused QKV projection)' if fused else ''}"
+                        f"{' (E4M3 pool: FP8 K/V pages + scales, FP8 attention)' if kv == 'fp8' else ''}"
+                        f": one layer-round, S={cfg.num_stages}+store, "
                         f"C={cfg.chunk_tokens}, heads={cfg.num_heads}x{cfg.head_dim}, "
                         f"anchor={cfg.anchor_chunks}, history={cfg.history_chunks}, "
                         f"page={cfg.page_tokens}, steady state",
@@ -544,6 +554,8 @@ def workload_config(cfg, n, fused=False):
 
 def main():
     args = parse()
+    if args.fused and args.kv == "fp8":
+        raise SystemExit("--fused publishes into bf16 pools only")
     ws, rank, local = dist_env()
     if ws > 1:
         import datetime
@@ -595,17 +607,22 @@ def main():
         value = whole_job_rate(res["flops"] * args.steps, res["ms"], ws) / 1e12
         att_tflops = res["flops"] / (res["att_ms"] * 1e-3) / 1e12
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        # An E4M3 contraction's peak: the measured bf16 peak times the nominal
+        # dense ratio fp8 / bf16 (4.5 / 2.25 PFLOP/s).
+        f8 = args.kv == "fp8"
+        ratio = 2.0 if f8 else 1.0
         pub_gbs = res["pbytes"] / (res["pub_ms"] * 1e-3) / 1e9
-        kfile = os.path.join(ROOT, "chunk_causal_wavefront_b200", "csrc", "attn_bf16.cu")
+        kfile = os.path.join(ROOT, "chunk_causal_wavefront_b200", "csrc", "attn_tc.cu")
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
-            "config": workload_config(cfg, ws, args.fused),
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if f8 else cfg.dtype,
+            "data": "synthetic",
+            "config": workload_config(cfg, ws, args.fused, args.kv),
             "rounds_per_s": ws * args.steps / (res["ms"] * 1e-3),
             "attention": {"ms_per_launch": res["att_ms"], "tflops": att_tflops,
-                          "pct_bf16_peak_burst": 100 * att_tflops / peaks["bf16_tflops"],
-                          "pct_bf16_peak_sustained": 100 * att_tflops / peak,
+                          "pct_peak_burst": 100 * att_tflops / (ratio * peaks["bf16_tflops"]),
+                          "pct_peak_sustained": 100 * att_tflops / (ratio * peak),
                           "flops_per_launch": res["flops"]},
             "publish": ({"ms_per_launch": res["pub_ms"], "gbs": pub_gbs,
                          "pct_hbm": 100 * pub_gbs / peaks["hbm_gbs"],
@@ -616,11 +633,12 @@ def main():
                          "pct_bf16_peak_burst": 100 * res["proj_flops"] / (res["pub_ms"] * 1e-3)
                          / 1e12 / peaks["bf16_tflops"],
                          "flops_per_launch": res["proj_flops"]}),
-            "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": peak,
-                         "unit": "TFLOP/s", "frac": att_tflops / peak,
-                         "traffic": read_traffic(kfile),
-                         "kernel": "attn_bf16_kernel",
-                         "peak_source": f"{src} bf16_tflops_sustained"},
+            "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": ratio * peak,
+                         "unit": "TFLOP/s", "frac": att_tflops / (ratio * peak),
+                         "traffic": read_traffic(kfile, "e4m3" if f8 else "bf16"),
+                         "kernel": "attn_tc_kernel<e4m3>" if f8 else "attn_tc_kernel<bf16>",
+                         "peak_source": f"{src} bf16_tflops_sustained"
+                                        + (" x 2 (nominal fp8/bf16 dense ratio)" if f8 else "")},
             "clocks": res["clocks"],
             "gpu_launches": 3 * args.steps,
         }

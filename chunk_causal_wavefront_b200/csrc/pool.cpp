@@ -53,6 +53,8 @@ struct Geometry {
   size_t rope_t_off = 0, rope_h_off = 0, rope_w_off = 0;
   size_t rope_t_n = 0, rope_h_n = 0, rope_w_n = 0;   // float2 entries
   size_t tags_off = 0, pages_off = 0, page_bytes = 0, total = 0;
+  size_t kv_scale_off = 0, q_scale_off = 0;           // FP8 pools only (else 0)
+  size_t kv_scale_per_layer = 0, q_scale_per_layer = 0;   // floats
 };
 
 wf_status validate(const wf_pool_config &c) {
@@ -63,7 +65,7 @@ wf_status validate(const wf_pool_config &c) {
   if (c.page_tokens < 1 || c.num_layers < 1 || c.max_rounds < 1) return WF_ERR_INVALID_ARG;
   if (c.num_pages < 0) return WF_ERR_INVALID_ARG;
   if (c.mask_mode != WF_MASK_WF && c.mask_mode != WF_MASK_RF) return WF_ERR_INVALID_ARG;
-  if (c.dtype == WF_DTYPE_BF16) {
+  if (c.dtype == WF_DTYPE_BF16 || c.dtype == WF_DTYPE_FP8_E4M3) {
     if (c.head_dim != 128 || c.page_tokens != 128) return WF_ERR_UNSUPPORTED;
   } else if (c.dtype == WF_DTYPE_F32) {
     if (c.head_dim % 4 != 0 || c.head_dim > 128) return WF_ERR_UNSUPPORTED;
@@ -99,7 +101,7 @@ wf_status geometry(const wf_pool_config &c, Geometry *g) {
       static_cast<int64_t>(c.num_stages + 1 + c.anchor_chunks + c.history_chunks) * g->npc;
   g->num_pages = c.num_pages == 0 ? min_pages : c.num_pages;
   if (g->num_pages < min_pages) return WF_ERR_OUT_OF_PAGES;
-  g->elt = c.dtype == WF_DTYPE_BF16 ? 2 : 4;
+  g->elt = c.dtype == WF_DTYPE_BF16 ? 2 : (c.dtype == WF_DTYPE_F32 ? 4 : 1);
   // Pool rows (one row = one token of one head of K or V) must fit int32 for
   // the tensor-map coordinates of the bf16 path.
   const int64_t rows = static_cast<int64_t>(c.num_layers) * g->num_pages * 2 * c.num_heads *
@@ -123,7 +125,16 @@ wf_status geometry(const wf_pool_config &c, Geometry *g) {
     off = align_up(off + g->rope_w_n * 8, 256);
   }
   g->tags_off = off;
-  off = align_up(off + static_cast<size_t>(c.num_layers) * g->num_pages * 4, 1024);
+  off = align_up(off + static_cast<size_t>(c.num_layers) * g->num_pages * 4, 256);
+  if (c.dtype == WF_DTYPE_FP8_E4M3) {
+    g->kv_scale_per_layer = static_cast<size_t>(g->num_pages) * 2 * c.num_heads;
+    g->q_scale_per_layer = static_cast<size_t>(c.num_stages + 1) * g->npc * c.num_heads;
+    g->kv_scale_off = off;
+    off = align_up(off + c.num_layers * g->kv_scale_per_layer * 4, 256);
+    g->q_scale_off = off;
+    off = align_up(off + c.num_layers * g->q_scale_per_layer * 4, 256);
+  }
+  off = align_up(off, 1024);
   g->pages_off = off;
   g->page_bytes = 2 * static_cast<size_t>(c.num_heads) * c.page_tokens * c.head_dim * g->elt;
   off += static_cast<size_t>(c.num_layers) * g->num_pages * g->page_bytes;
@@ -146,15 +157,21 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-bool encode_bf16_map(CUtensorMap *map, void *base, int rank, const cuuint64_t *dims,
-                     const cuuint64_t *strides_bytes, const cuuint32_t *box) {
+// 128-byte-swizzled tiled map over bf16 elements or raw bytes (E4M3 codes).
+bool encode_map(CUtensorMap *map, CUtensorMapDataType type, void *base, int rank,
+                const cuuint64_t *dims, const cuuint64_t *strides_bytes, const cuuint32_t *box) {
   auto fn = get_encode();
   if (!fn) return false;
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides_bytes, box,
+  CUresult r = fn(map, type, rank, base, dims, strides_bytes, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_bf16_map(CUtensorMap *map, void *base, int rank, const cuuint64_t *dims,
+                     const cuuint64_t *strides_bytes, const cuuint32_t *box) {
+  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box);
 }
 
 }  // namespace
@@ -174,7 +191,7 @@ struct wf_pool {
   std::vector<int32_t> anchor_pages;
   std::deque<std::pair<int, std::vector<int32_t>>> history;
   std::vector<Position> layout;                   // current ordered context
-  CUtensorMap kv_map;                             // bf16 pages, 2D rows x d
+  CUtensorMap kv_map;                             // bf16 / E4M3 pages, 2D rows x d
 };
 
 namespace {
@@ -354,13 +371,16 @@ wf_status wf_kv_pool_create(const wf_pool_config *cfg, void *dev_mem, size_t byt
       delete p;
       return WF_ERR_CUDA;
     }
-    if (cfg->dtype == WF_DTYPE_BF16) {
+    if (cfg->dtype == WF_DTYPE_BF16 || cfg->dtype == WF_DTYPE_FP8_E4M3) {
+      // One pool row = one token of one head of K or V: 128 elements.
+      const bool f8 = cfg->dtype == WF_DTYPE_FP8_E4M3;
       const cuuint64_t rows = static_cast<cuuint64_t>(cfg->num_layers) * g.num_pages * 2 *
                               cfg->num_heads * cfg->page_tokens;
       const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cfg->head_dim), rows};
-      const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cfg->head_dim) * 2};
-      const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(cfg->page_tokens)};
-      if (!encode_bf16_map(&p->kv_map, p->dev + g.pages_off, 2, dims, strides, box)) {
+      const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cfg->head_dim) * g.elt};
+      const cuuint32_t box[2] = {f8 ? 128u : 64u, static_cast<cuuint32_t>(cfg->page_tokens)};
+      if (!encode_map(&p->kv_map, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                      p->dev + g.pages_off, 2, dims, strides, box)) {
         delete p;
         return WF_ERR_CUDA;
       }
@@ -398,8 +418,16 @@ wf_status wf_publish_kv(wf_pool *p, int32_t layer, const void *q, const void *k,
   pp.rope = c.rope; pp.F = c.frames_per_chunk; pp.gh = c.grid_h; pp.gw = c.grid_w;
   pp.split0 = c.rope_split[0]; pp.split1 = c.rope_split[1]; pp.split2 = c.rope_split[2];
   pp.live = live_slots(p);
+  if (c.dtype == WF_DTYPE_FP8_E4M3) {
+    pp.kv_scale = reinterpret_cast<float *>(p->dev + p->g.kv_scale_off) +
+                  static_cast<size_t>(layer) * p->g.kv_scale_per_layer;
+    pp.q_scale = reinterpret_cast<float *>(p->dev + p->g.q_scale_off) +
+                 static_cast<size_t>(layer) * p->g.q_scale_per_layer;
+  }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = c.dtype == WF_DTYPE_BF16 ? launch_publish_bf16(pp, cs) : launch_publish_f32(pp, cs);
+  cudaError_t e = c.dtype == WF_DTYPE_BF16 ? launch_publish_bf16(pp, cs)
+                  : c.dtype == WF_DTYPE_F32 ? launch_publish_f32(pp, cs)
+                                            : launch_publish_fp8(pp, cs);
   return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 
@@ -428,23 +456,37 @@ wf_status wf_round_attention(wf_pool *p, int32_t layer, const void *q_rot, void 
   ap.live = live_slots(p);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (c.dtype == WF_DTYPE_BF16) {
-    CUtensorMap qmap;
+  if (c.dtype == WF_DTYPE_BF16 || c.dtype == WF_DTYPE_FP8_E4M3) {
+    const bool f8 = c.dtype == WF_DTYPE_FP8_E4M3;
+    // [S+1][C][heads][d] activations; q_rot in the pool's element type, out bf16.
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(c.head_dim),
                                 static_cast<cuuint64_t>(c.num_heads),
                                 static_cast<cuuint64_t>(c.chunk_tokens),
                                 static_cast<cuuint64_t>(c.num_stages + 1)};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(c.head_dim) * 2,
-                                   static_cast<cuuint64_t>(c.head_dim) * 2 * c.num_heads,
-                                   static_cast<cuuint64_t>(c.head_dim) * 2 * c.num_heads *
-                                       c.chunk_tokens};
-    const cuuint32_t box[4] = {64, 1, 128, 1};
-    if (!encode_bf16_map(&qmap, const_cast<void *>(q_rot), 4, dims, strides, box))
+    auto strides_of = [&](cuuint64_t elt, cuuint64_t *st) {
+      st[0] = static_cast<cuuint64_t>(c.head_dim) * elt;
+      st[1] = st[0] * c.num_heads;
+      st[2] = st[1] * c.chunk_tokens;
+    };
+    cuuint64_t qstr[3], ostr[3];
+    strides_of(p->g.elt, qstr);
+    strides_of(2, ostr);
+    CUtensorMap qmap, omap;
+    const cuuint32_t qbox[4] = {f8 ? 128u : 64u, 1, 128, 1};
+    if (!encode_map(&qmap, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                    const_cast<void *>(q_rot), 4, dims, qstr, qbox))
       return WF_ERR_CUDA;
-    CUtensorMap omap;
     const cuuint32_t obox[4] = {64, 1, 32, 1};
-    if (!encode_bf16_map(&omap, out, 4, dims, strides, obox)) return WF_ERR_CUDA;
-    e = launch_attention_bf16(ap, &qmap, &p->kv_map, &omap, cs);
+    if (!encode_bf16_map(&omap, out, 4, dims, ostr, obox)) return WF_ERR_CUDA;
+    if (f8) {
+      ap.kv_scale = reinterpret_cast<const float *>(p->dev + p->g.kv_scale_off) +
+                    static_cast<size_t>(layer) * p->g.kv_scale_per_layer;
+      ap.q_scale = reinterpret_cast<const float *>(p->dev + p->g.q_scale_off) +
+                   static_cast<size_t>(layer) * p->g.q_scale_per_layer;
+      e = launch_attention_fp8(ap, &qmap, &p->kv_map, &omap, cs);
+    } else {
+      e = launch_attention_bf16(ap, &qmap, &p->kv_map, &omap, cs);
+    }
   } else {
     e = launch_attention_f32(ap, cs);
   }
@@ -562,6 +604,8 @@ wf_status wf_pool_get_geometry(const wf_pool *p, wf_pool_geometry *geom) {
   geom->pages_offset = p->g.pages_off;
   geom->page_bytes = p->g.page_bytes;
   geom->total_bytes = p->g.total;
+  geom->kv_scale_offset = p->g.kv_scale_off;
+  geom->q_scale_offset = p->g.q_scale_off;
   return WF_OK;
 }
 

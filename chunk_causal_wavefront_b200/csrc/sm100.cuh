@@ -283,5 +283,79 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool b_mn_m
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// D[tmem] (+)= A[smem] * B[smem] for 8-bit floats (kind::f8f6f4, K = 32 per
+// instruction), descriptors given as (lo, hi) words.
+__device__ __forceinline__ void mma_f8_ss2(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                           uint32_t hi, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "mov.b64 da, {%1, %3};\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem] for 8-bit floats; A holds four 8-bit values
+// per 32-bit TMEM column (element 4c + i in byte i of column c).
+__device__ __forceinline__ void mma_f8_ts2(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                           uint32_t hi, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor for kind::f8f6f4 with E4M3 A/B (format code 0) and
+// fp32 accumulation; same field positions as make_idesc_bf16.
+__host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N, bool b_mn_major) {
+  return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// 32 lanes x 8 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
+// Two fp32 values rounded to nearest-even E4M3 (saturating to +-448): a in
+// byte 0, b in byte 1 of the low half of the result.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float a, float b) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 h;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h, %2, %1;\n\t"
+      "cvt.u32.u16 %0, h;\n\t}"
+      : "=r"(r)
+      : "f"(a), "f"(b));
+  return r;
+}
+
+// Bytes 0-1 of lo and bytes 0-1 of hi as one 32-bit word.
+__device__ __forceinline__ uint32_t join16(uint32_t lo, uint32_t hi) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+
+// Four fp32 values rounded to nearest-even E4M3 (saturating to +-448), packed
+// with a in byte 0, b in byte 1, c in byte 2 and d in byte 3.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
+}
+
 }  // namespace sm100
 }  // namespace wf

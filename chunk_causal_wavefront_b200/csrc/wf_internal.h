@@ -46,6 +46,8 @@ struct PublishParams {
   const int32_t *table;       // device page table
   int32_t *status;            // sticky status word
   const float2 *rope_t, *rope_h, *rope_w;  // (cos, sin) per position x pair
+  float *kv_scale;            // FP8 pool: this layer's [num_pages][2][heads] block scales
+  float *q_scale;             // FP8 pool: this layer's [S+1][npc][heads] query-tile scales
   int32_t S1, C, Hh, d, P, npc, num_pages;
   int32_t rope, F, gh, gw, split0, split1, split2;
   LiveSlots live;
@@ -59,7 +61,9 @@ struct AttnParams {
   const int32_t *table;
   int32_t *status;
   int32_t S1, C, Hh, d, P, npc, num_pages, n_pos;
-  int64_t layer_row0;         // first pool row of this layer (bf16 tensor map)
+  int64_t layer_row0;         // first pool row of this layer (pool tensor map)
+  const float *kv_scale;      // FP8 pool: this layer's [num_pages][2][heads] block scales
+  const float *q_scale;       // FP8 pool: this layer's [S+1][npc][heads] query-tile scales
   float scale_log2;           // log2(e) / sqrt(d)
   float scale;                // 1 / sqrt(d)
   LiveSlots live;
@@ -80,6 +84,7 @@ struct ProjectParams {
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_publish_bf16(const PublishParams &p, cudaStream_t st);
 cudaError_t launch_publish_f32(const PublishParams &p, cudaStream_t st);
+cudaError_t launch_publish_fp8(const PublishParams &p, cudaStream_t st);
 cudaError_t launch_attention_f32(const AttnParams &p, cudaStream_t st);
 // The bf16 tensor-core path takes the encoded tensor maps (opaque 128-byte
 // CUtensorMap objects) of q_rot (box 64 x 1 x 128 rows), the pool's K/V pages
@@ -87,6 +92,10 @@ cudaError_t launch_attention_f32(const AttnParams &p, cudaStream_t st);
 cudaError_t launch_attention_bf16(const AttnParams &p, const void *tmap_q,
                                   const void *tmap_kv, const void *tmap_out,
                                   cudaStream_t st);
+// The FP8 path: q_rot and the pages are E4M3 bytes (q box 128 x 1 x 128 rows,
+// page box 128 x 128), out is bf16 (box 64 x 1 x 32 rows).
+cudaError_t launch_attention_fp8(const AttnParams &p, const void *tmap_q,
+                                 const void *tmap_kv, const void *tmap_out, cudaStream_t st);
 // Fused QKV projection: tensor maps of x (3D: hidden x C x S+1, box 64 x 256 x 1)
 // and w_qkv (2D: hidden x 3*hidden, box 64 x 256).
 cudaError_t launch_project_bf16(const ProjectParams &p, const void *tmap_x, const void *tmap_w,

@@ -12,7 +12,10 @@ import torch
 from . import wf as _wf
 from .wf import WfError, WfPoolConfig
 
-_DTYPES = {"bf16": (_wf.WF_DTYPE_BF16, torch.bfloat16), "f32": (_wf.WF_DTYPE_F32, torch.float32)}
+# pool dtype -> (C enum, element type of the pages and of q_rot)
+_DTYPES = {"bf16": (_wf.WF_DTYPE_BF16, torch.bfloat16), "f32": (_wf.WF_DTYPE_F32, torch.float32),
+           "fp8": (_wf.WF_DTYPE_FP8_E4M3, torch.uint8)}
+_ELEMENT = {code: t for code, t in _DTYPES.values()}
 
 
 def make_config(*, num_stages: int, chunk_tokens: int, num_heads: int, head_dim: int,
@@ -60,7 +63,10 @@ class KVPool:
         self.cfg = cfg
         self.nbytes = _wf.wf_kv_pool_bytes(cfg)
         self.device = None if device is None else torch.device(device)
-        self.dtype = torch.bfloat16 if cfg.dtype == _wf.WF_DTYPE_BF16 else torch.float32
+        # element type of the pages and of q_rot (E4M3 codes as uint8 for FP8
+        # pools); q, k, v inputs and out are bf16 for bf16 and FP8 pools
+        self.dtype = _ELEMENT[cfg.dtype]
+        self.io_dtype = torch.float32 if cfg.dtype == _wf.WF_DTYPE_F32 else torch.bfloat16
         self.mem = None
         if self.device is not None:
             if mem is not None:
@@ -120,11 +126,29 @@ class KVPool:
     def pages_view(self) -> torch.Tensor:
         """The page region as [layers][num_pages][2][heads][P][d] (K = 0, V = 1)."""
         g, c = self.geometry, self.cfg
-        elt = 2 if self.dtype == torch.bfloat16 else 4
         n = c.num_layers * g.num_pages * g.page_bytes
         raw = self.mem[g.pages_offset:g.pages_offset + n]
         return raw.view(self.dtype).view(c.num_layers, g.num_pages, 2, c.num_heads,
                                          c.page_tokens, c.head_dim)
+
+    def kv_scales_view(self) -> torch.Tensor:
+        """FP8 pools: the block scales as [layers][num_pages][2][heads] fp32."""
+        g, c = self.geometry, self.cfg
+        if c.dtype != _wf.WF_DTYPE_FP8_E4M3:
+            raise ValueError("only FP8 pools carry scales")
+        n = c.num_layers * g.num_pages * 2 * c.num_heads * 4
+        raw = self.mem[g.kv_scale_offset:g.kv_scale_offset + n]
+        return raw.view(torch.float32).view(c.num_layers, g.num_pages, 2, c.num_heads)
+
+    def q_scales_view(self) -> torch.Tensor:
+        """FP8 pools: q_rot's tile scales as [layers][S+1][pages_per_chunk][heads] fp32."""
+        g, c = self.geometry, self.cfg
+        if c.dtype != _wf.WF_DTYPE_FP8_E4M3:
+            raise ValueError("only FP8 pools carry scales")
+        n = c.num_layers * (c.num_stages + 1) * g.pages_per_chunk * c.num_heads * 4
+        raw = self.mem[g.q_scale_offset:g.q_scale_offset + n]
+        return raw.view(torch.float32).view(c.num_layers, c.num_stages + 1, g.pages_per_chunk,
+                                            c.num_heads)
 
     def tags_view(self) -> torch.Tensor:
         g, c = self.geometry, self.cfg

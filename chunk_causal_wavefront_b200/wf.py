@@ -24,6 +24,7 @@ WF_ERR_UNSUPPORTED = 7
 WF_ERR_TIMEOUT = 8
 WF_DTYPE_BF16 = 0
 WF_DTYPE_F32 = 1
+WF_DTYPE_FP8_E4M3 = 2
 WF_ROPE_OFF = 0
 WF_ROPE_3D = 1
 WF_MASK_WF = 0
@@ -58,6 +59,7 @@ class WfPoolGeometry(ctypes.Structure):
         ("max_positions", ctypes.c_int32), ("status_offset", ctypes.c_size_t),
         ("tags_offset", ctypes.c_size_t), ("pages_offset", ctypes.c_size_t),
         ("page_bytes", ctypes.c_size_t), ("total_bytes", ctypes.c_size_t),
+        ("kv_scale_offset", ctypes.c_size_t), ("q_scale_offset", ctypes.c_size_t),
     ]
 
 

@@ -20,7 +20,8 @@
  *   - Pointers named q, k, v, q_rot, out and dev_mem are DEVICE pointers on the
  *     current CUDA device; config structs and page_order are HOST pointers.
  *   - Activations are laid out [S+1][C][num_heads][head_dim], row-major, in the
- *     pool's dtype (bf16 or fp32): slot-major, then token, head, dimension.
+ *     pool's dtype (bf16 or fp32; FP8 pools: see WF_DTYPE_FP8_E4M3): slot-major,
+ *     then token, head, dimension.
  *     Slot s < S holds the chunk at denoising stage s; slot S is the store.
  *   - Every call that takes a stream enqueues its device work on that stream
  *     (NULL = legacy default stream) and returns without synchronising, except
@@ -59,7 +60,20 @@ typedef enum {
   WF_ERR_TIMEOUT = 8        /* a bounded device-side wait ran out (kernel gave up) */
 } wf_status;
 
-enum { WF_DTYPE_BF16 = 0, WF_DTYPE_F32 = 1 };
+/* Storage / compute type of a pool.
+ * BF16: pages, q, k, v, q_rot and out are bf16; tensor-core attention.
+ * F32:  all fp32; CUDA-core attention.
+ * FP8_E4M3: the K/V payload plus scale factors of Appendix Table 8 ("FP8 K/V
+ *   communication"), with 8-bit attention operands as in the Sage backends of
+ *   Tables 4-6. Pages hold E4M3 codes (1 byte per element, round to nearest
+ *   even); every (page, K|V, head) block of 128 x d codes has a power-of-two
+ *   fp32 scale 2^e, e the smallest integer with amax * 2^-e <= 448 (clamped
+ *   below at -100). wf_publish_kv reads bf16 q, k, v, rotates q and k in fp32
+ *   (each product and sum rounded once), and writes q_rot as E4M3 codes
+ *   [S+1][C][heads][d] with one scale per (slot, 128-row tile, head) kept in
+ *   the pool. wf_round_attention reads those codes and scales and writes bf16
+ *   out. Needs head_dim 128 and page_tokens 128. */
+enum { WF_DTYPE_BF16 = 0, WF_DTYPE_F32 = 1, WF_DTYPE_FP8_E4M3 = 2 };
 enum { WF_ROPE_OFF = 0, WF_ROPE_3D = 1 };
 /* Which (query slot, key slot) pairs are visible.
  * WF: M_WF(s, j) = 1[j >= s] (Method section of the hyper.ai summary), plus
@@ -82,7 +96,7 @@ typedef struct {
   int32_t history_chunks;  /* H, bounded clean history window, 0..WF_MAX_HISTORY */
   int32_t page_tokens;     /* P, tokens per page; bf16 attention: 128 */
   int32_t num_layers;      /* layers sharing the page table (one pool region each) */
-  int32_t dtype;           /* WF_DTYPE_BF16 or WF_DTYPE_F32 */
+  int32_t dtype;           /* WF_DTYPE_BF16, WF_DTYPE_F32 or WF_DTYPE_FP8_E4M3 */
   int32_t rope;            /* WF_ROPE_OFF or WF_ROPE_3D */
   int32_t frames_per_chunk;/* F: latent frames per chunk (3D rotary only) */
   int32_t grid_h, grid_w;  /* patch grid per frame; C == F * grid_h * grid_w */
@@ -105,6 +119,9 @@ typedef struct {
   size_t pages_offset;      /* [num_layers][num_pages][2 (K,V)][heads][P][d] */
   size_t page_bytes;        /* bytes of one (layer, page): 2 * heads * P * d * elt */
   size_t total_bytes;       /* == wf_kv_pool_bytes */
+  size_t kv_scale_offset;   /* FP8: fp32 [num_layers][num_pages][2 (K,V)][heads]; else 0 */
+  size_t q_scale_offset;    /* FP8: fp32 [num_layers][S+1][pages_per_chunk][heads]
+                               (scale of q_rot rows [128 t, 128 t + 128)); else 0 */
 } wf_pool_geometry;
 
 /* Bytes of device memory a pool with this config needs (the caller allocates
@@ -135,6 +152,8 @@ wf_status wf_kv_pool_create(const wf_pool_config *cfg, void *dev_mem, size_t byt
  *   q, k, v : inputs, [S+1][C][heads][d]; rows of slots that are not live in
  *             this round are not read.
  *   q_rot   : output, same layout; only live slots' rows are written.
+ * FP8_E4M3 pools: q, k, v are bf16; q_rot receives E4M3 codes (1 byte per
+ * element) and the pool records the block scales of q_rot, K and V.
  * Pointers must be 16-byte aligned; q_rot must not alias q, k or v. */
 wf_status wf_publish_kv(wf_pool *pool, int32_t layer, const void *q, const void *k,
                         const void *v, void *q_rot, wf_stream_t stream);
@@ -150,7 +169,10 @@ wf_status wf_publish_kv(wf_pool *pool, int32_t layer, const void *q, const void 
  *   q_rot : [S+1][C][heads][d] rotated queries (as written by wf_publish_kv);
  *   out   : [S+1][C][heads][d]; rows of non-live slots are left untouched.
  * bf16 pools need head_dim == 128 and page_tokens == 128 (tensor-core path);
- * fp32 pools run a CUDA-core path. Pointers must be 16-byte aligned. */
+ * fp32 pools run a CUDA-core path. FP8_E4M3 pools read q_rot codes as written
+ * by wf_publish_kv in this round for this layer (their scales live in the
+ * pool), run E4M3 tensor-core MMAs (P rounded to E4M3 too) and write bf16 out.
+ * Pointers must be 16-byte aligned. */
 wf_status wf_round_attention(wf_pool *pool, int32_t layer, const void *q_rot, void *out,
                              wf_stream_t stream);
 
@@ -168,7 +190,7 @@ wf_status wf_round_attention(wf_pool *pool, int32_t layer, const void *q_rot, vo
  *           (row f holds the weights of output feature f).
  *   q_rot : [S+1][C][heads][d] bf16; only live slots' rows are written.
  * bf16 pools only, with head_dim 128, page_tokens 128 and hidden a multiple of
- * 256 (WF_ERR_UNSUPPORTED otherwise). Pointers must be 16-byte aligned. */
+ * 256 (WF_ERR_UNSUPPORTED otherwise, FP8 pools included). Pointers must be 16-byte aligned. */
 wf_status wf_project_publish(wf_pool *pool, int32_t layer, const void *x, const void *w_qkv,
                              void *q_rot, wf_stream_t stream);
 

@@ -55,6 +55,29 @@ def test_pool_bytes_and_geometry():
     pool.close()
 
 
+def test_fp8_pool_geometry():
+    """FP8 pools: 1-byte pages (half of bf16) plus fp32 block scales for every
+    (layer, page, K|V, head) and every (layer, slot, query tile, head)."""
+    cfg = wf_inputs.CONFIGS["wan13b_bf16"]
+    c = pool_config(cfg, dtype="fp8", num_layers=3)
+    pool = wfb.KVPool(c)
+    g = pool.geometry
+    assert g.page_bytes == 2 * 12 * 128 * 128
+    assert g.pages_offset % 1024 == 0 and g.kv_scale_offset % 256 == 0
+    assert g.tags_offset < g.kv_scale_offset < g.q_scale_offset < g.pages_offset
+    assert g.q_scale_offset - g.kv_scale_offset >= 3 * g.num_pages * 2 * 12 * 4
+    assert g.pages_offset - g.q_scale_offset >= 3 * 5 * 37 * 12 * 4
+    assert g.total_bytes >= g.pages_offset + 3 * g.num_pages * g.page_bytes
+    bf = wfb.KVPool(pool_config(cfg, num_layers=3)).geometry
+    assert bf.kv_scale_offset == 0 and bf.q_scale_offset == 0
+    assert bf.page_bytes == 2 * g.page_bytes
+    pool.close()
+    for over in (dict(head_dim=64), dict(page_tokens=64)):
+        with pytest.raises(W.WfError) as e:
+            W.wf_kv_pool_bytes(pool_config(cfg, dtype="fp8", **over))
+        assert e.value.status == W.WF_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("over,err", [
     (dict(num_stages=0), W.WF_ERR_INVALID_ARG),
     (dict(num_stages=17), W.WF_ERR_INVALID_ARG),
