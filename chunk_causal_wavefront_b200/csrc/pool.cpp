@@ -169,6 +169,18 @@ bool encode_map(CUtensorMap *map, CUtensorMapDataType type, void *base, int rank
   return r == CUDA_SUCCESS;
 }
 
+// Unswizzled tiled map over bf16 elements (rows of the box land contiguously).
+bool encode_plain_bf16_map(CUtensorMap *map, void *base, int rank, const cuuint64_t *dims,
+                           const cuuint64_t *strides_bytes, const cuuint32_t *box) {
+  auto fn = get_encode();
+  if (!fn) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides_bytes, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool encode_bf16_map(CUtensorMap *map, void *base, int rank, const cuuint64_t *dims,
                      const cuuint64_t *strides_bytes, const cuuint32_t *box) {
   return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box);
@@ -425,9 +437,25 @@ wf_status wf_publish_kv(wf_pool *p, int32_t layer, const void *q, const void *k,
                  static_cast<size_t>(layer) * p->g.q_scale_per_layer;
   }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = c.dtype == WF_DTYPE_BF16 ? launch_publish_bf16(pp, cs)
-                  : c.dtype == WF_DTYPE_F32 ? launch_publish_f32(pp, cs)
-                                            : launch_publish_fp8(pp, cs);
+  cudaError_t e;
+  if (c.dtype == WF_DTYPE_FP8_E4M3) {
+    // [S+1][C][heads][d] bf16; one box is a 128-row tile of one head.
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(c.head_dim),
+                                static_cast<cuuint64_t>(c.num_heads),
+                                static_cast<cuuint64_t>(c.chunk_tokens),
+                                static_cast<cuuint64_t>(c.num_stages + 1)};
+    const cuuint64_t row = static_cast<cuuint64_t>(c.head_dim) * 2;
+    const cuuint64_t strides[3] = {row, row * c.num_heads, row * c.num_heads * c.chunk_tokens};
+    const cuuint32_t box[4] = {128, 1, 128, 1};
+    CUtensorMap mq, mk, mv;
+    if (!encode_plain_bf16_map(&mq, const_cast<void *>(q), 4, dims, strides, box) ||
+        !encode_plain_bf16_map(&mk, const_cast<void *>(k), 4, dims, strides, box) ||
+        !encode_plain_bf16_map(&mv, const_cast<void *>(v), 4, dims, strides, box))
+      return WF_ERR_CUDA;
+    e = launch_publish_fp8(pp, &mq, &mk, &mv, cs);
+  } else {
+    e = c.dtype == WF_DTYPE_BF16 ? launch_publish_bf16(pp, cs) : launch_publish_f32(pp, cs);
+  }
   return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 

@@ -84,7 +84,10 @@ struct ProjectParams {
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_publish_bf16(const PublishParams &p, cudaStream_t st);
 cudaError_t launch_publish_f32(const PublishParams &p, cudaStream_t st);
-cudaError_t launch_publish_fp8(const PublishParams &p, cudaStream_t st);
+// The FP8 publish takes unswizzled tensor maps of q, k and v over
+// [S+1][C][heads][d] bf16 with a box of 128 dims x 1 head x 128 rows.
+cudaError_t launch_publish_fp8(const PublishParams &p, const void *tmap_q, const void *tmap_k,
+                               const void *tmap_v, cudaStream_t st);
 cudaError_t launch_attention_f32(const AttnParams &p, cudaStream_t st);
 // The bf16 tensor-core path takes the encoded tensor maps (opaque 128-byte
 // CUtensorMap objects) of q_rot (box 64 x 1 x 128 rows), the pool's K/V pages
