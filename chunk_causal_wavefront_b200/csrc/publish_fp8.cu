@@ -51,8 +51,8 @@ constexpr uint32_t kTensorBytes = kRows * 128 * 2;      // one bf16 tile, 32 KB
 constexpr uint32_t kStageBytes = 3 * kTensorBytes;      // q, k, v
 constexpr uint32_t kOffBars = 2 * kStageBytes;          // two stages
 constexpr uint32_t kOffRed = kOffBars + 64;             // [3][kWarps] block maxima
-constexpr uint32_t kOffPos = kOffRed + 3 * kWarps * 4;  // [3][kRows] rotary t, y, x
-constexpr uint32_t kSmemBytes = kOffPos + 3 * kRows * 4 + 1024;
+constexpr uint32_t kOffPos = kOffRed + 3 * kWarps * 4;  // [kRows][4] rotary table offsets
+constexpr uint32_t kSmemBytes = kOffPos + 4 * kRows * 4 + 1024;
 
 // Smallest e with amax * 2^-e <= 448 = 1.75 * 2^8, clamped below at -100:
 // for amax = f * 2^E (f in [1, 2)), e = E - 8 if f <= 1.75, else E - 7.
@@ -169,26 +169,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBars);   // [2]
   float *red = reinterpret_cast<float *>(smem + kOffRed);
-  int32_t *pos = reinterpret_cast<int32_t *>(smem + kOffPos);      // t[128], y[128], x[128]
+  int32_t *pos = reinterpret_cast<int32_t *>(smem + kOffPos);      // [row][t, h, w, -]
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBars + 16);
   const int nblk = p.live.n * p.npc * p.Hh;
   const int G = gridDim.x;
   const int cv = threadIdx.x & (kTPR - 1);        // 16-byte vector of the head row
   const int r0 = threadIdx.x / kTPR;              // first row of this thread
   const Ctx ctx{full, abort_flag, p.status};
-  // Rotary (cos, sin) rows of this thread's 4 pairs (pairs 4 cv .. 4 cv + 3):
-  // pair pr lies in band t, h or w; its entry for a row at band position x is
-  // ctab[i][x * cmul[i]], x read from pos[cpos[i] + row].
-  const float2 *ctab[4] = {nullptr, nullptr, nullptr, nullptr};
-  int cmul[4] = {0, 0, 0, 0}, cpos[4] = {0, 0, 0, 0};
+  // Rotary (cos, sin) entries of this thread's 4 pairs (pairs 4 cv .. 4 cv + 3):
+  // pair pr lies in band t, h or w (band index b); its entry for row r is
+  // rope_t[o + pos[4 r + b]], o the pair's offset from the t table (the three
+  // tables share the pool buffer) and pos the row's position in each band
+  // times that band's pair count. ctab[i] packs 4 o + b.
+  const int h0 = p.split0 >> 1, h1 = p.split1 >> 1, h2 = p.split2 >> 1;
+  int ctab[4] = {0, 0, 0, 0};
   if (p.rope) {
-    const int h0 = p.split0 >> 1, h1 = p.split1 >> 1, h2 = p.split2 >> 1;
+    const int oh = static_cast<int>(p.rope_h - p.rope_t), ow = static_cast<int>(p.rope_w - p.rope_t);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int pr = cv * 4 + i;
-      if (pr < h0) { ctab[i] = p.rope_t + pr; cmul[i] = h0; cpos[i] = 0; }
-      else if (pr < h0 + h1) { ctab[i] = p.rope_h + (pr - h0); cmul[i] = h1; cpos[i] = kRows; }
-      else { ctab[i] = p.rope_w + (pr - h0 - h1); cmul[i] = h2; cpos[i] = 2 * kRows; }
+      if (pr < h0) ctab[i] = 4 * pr;
+      else if (pr < h0 + h1) ctab[i] = 4 * (oh + pr - h0) + 1;
+      else ctab[i] = 4 * (ow + pr - h0 - h1) + 2;
     }
   }
 
@@ -231,9 +233,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int n = j * kRows + threadIdx.x;
       if (n >= p.C) n = 0;
       const int hw = p.gh * p.gw, f = n / hw, yx = n - f * hw, y = yx / p.gw;
-      pos[threadIdx.x] = p.F * p.live.chunk[li] + f;
-      pos[kRows + threadIdx.x] = y;
-      pos[2 * kRows + threadIdx.x] = yx - y * p.gw;
+      pos[4 * threadIdx.x] = (p.F * p.live.chunk[li] + f) * h0;
+      pos[4 * threadIdx.x + 1] = y * h1;
+      pos[4 * threadIdx.x + 2] = (yx - y * p.gw) * h2;
     }
     // The n-th use of a stage waits for its n-th fill: parity (i / 2) & 1.
     const bool ok = __all_sync(0xffffffffu, wait_bar(ctx, stage, (i >> 1) & 1));
@@ -255,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.rope && j * kRows + r < p.C) {
         float2 cs[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) cs[c] = __ldg(ctab[c] + pos[cpos[c] + r] * cmul[c]);
+        for (int c = 0; c < 4; ++c) cs[c] = __ldg(p.rope_t + (ctab[c] >> 2) + pos[4 * r + (ctab[c] & 3)]);
         rotate8(xq[ps], cs);
         rotate8(xk[ps], cs);
       }
