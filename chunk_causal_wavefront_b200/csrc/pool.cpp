@@ -551,8 +551,9 @@ wf_status wf_project_publish(wf_pool *p, int32_t layer, const void *x, const voi
   pp.hidden = hidden;
   pp.rope = c.rope; pp.F = c.frames_per_chunk; pp.gh = c.grid_h; pp.gw = c.grid_w;
   pp.split0 = c.rope_split[0]; pp.split1 = c.rope_split[1]; pp.split2 = c.rope_split[2];
+  pp.layer_row0 = static_cast<int64_t>(layer) * p->g.num_pages * 2 * c.num_heads * c.page_tokens;
   pp.live = live_slots(p);
-  CUtensorMap xmap, wmap;
+  CUtensorMap xmap, wmap, qmap, kvmap;
   const cuuint64_t xd[3] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(c.chunk_tokens),
                             static_cast<cuuint64_t>(c.num_stages + 1)};
   const cuuint64_t xs[2] = {static_cast<cuuint64_t>(hidden) * 2,
@@ -563,7 +564,23 @@ wf_status wf_project_publish(wf_pool *p, int32_t layer, const void *x, const voi
   const cuuint64_t ws[1] = {static_cast<cuuint64_t>(hidden) * 2};
   const cuuint32_t wb[2] = {64, 256};
   if (!encode_bf16_map(&wmap, const_cast<void *>(w_qkv), 2, wd, ws, wb)) return WF_ERR_CUDA;
-  cudaError_t e = launch_project_bf16(pp, &xmap, &wmap, reinterpret_cast<cudaStream_t>(stream));
+  // Epilogue stores: q_rot [S+1][C][heads][d] and the pool's K/V rows, 32 rows per box.
+  const cuuint64_t qd[4] = {static_cast<cuuint64_t>(c.head_dim), static_cast<cuuint64_t>(c.num_heads),
+                            static_cast<cuuint64_t>(c.chunk_tokens),
+                            static_cast<cuuint64_t>(c.num_stages + 1)};
+  const cuuint64_t qs[3] = {static_cast<cuuint64_t>(c.head_dim) * 2,
+                            static_cast<cuuint64_t>(c.head_dim) * 2 * c.num_heads,
+                            static_cast<cuuint64_t>(c.head_dim) * 2 * c.num_heads * c.chunk_tokens};
+  const cuuint32_t qb[4] = {64, 1, 32, 1};
+  if (!encode_bf16_map(&qmap, q_rot, 4, qd, qs, qb)) return WF_ERR_CUDA;
+  const cuuint64_t kd[2] = {static_cast<cuuint64_t>(c.head_dim),
+                            static_cast<cuuint64_t>(c.num_layers) * p->g.num_pages * 2 *
+                                c.num_heads * c.page_tokens};
+  const cuuint64_t ks[1] = {static_cast<cuuint64_t>(c.head_dim) * 2};
+  const cuuint32_t kb[2] = {64, 32};
+  if (!encode_bf16_map(&kvmap, p->dev + p->g.pages_off, 2, kd, ks, kb)) return WF_ERR_CUDA;
+  cudaError_t e = launch_project_bf16(pp, &xmap, &wmap, &qmap, &kvmap,
+                                      reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 

@@ -21,10 +21,15 @@
 //                      k-step (one per page of the tile), fp32 accumulation
 //                      in TMEM columns [0, 256) and [256, 512);
 //   warps 0-7          epilogue, one warpgroup per page: thread r owns token r
-//                      of its page (TMEM lane r), loads its row 32 columns at a
-//                      time, rotates q and k pairs in fp32 with the pool's
-//                      (cos, sin) tables, rounds once to bf16 and stores
-//                      64-byte pieces to q_rot or to the page row.
+//                      of its page (TMEM lane r) and drains its row 32 columns
+//                      at a time (the next piece's TMEM load and (cos, sin)
+//                      loads in flight), rotates q and k pairs in fp32 with the
+//                      pool's tables, rounds once to bf16 and stages the rows in
+//                      the drained operand ring (128-byte swizzle). Each warp
+//                      then writes its 32 rows with TMA stores: q_rot through
+//                      the activation map, K and V into the page rows; the
+//                      first 64-dimension half is stored while the second is
+//                      computed.
 // Order of CTAs: feature tiles fastest, so consecutive CTAs share the x tile
 // and sweep w (14 MB for the 1.3B shape), which both stay in L2.
 #include <cuda.h>
@@ -47,6 +52,11 @@ constexpr int kStages = 3;
 constexpr uint32_t kABytes = kGM * kGK * 2;   // 32 KB
 constexpr uint32_t kBBytes = kGN * kGK * 2;   // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
+// Epilogue staging in the drained operand ring: per page of the tile, two
+// heads x two 64-dimension halves of 128 rows x 128 bytes.
+constexpr uint32_t kHalfStage = kPage * 128;                    // 16 KB
+constexpr uint32_t kHeadStage = 2 * kHalfStage;                 // 32 KB
+static_assert(2 * 2 * kHeadStage <= kStages * kStageBytes, "epilogue staging fits the ring");
 constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -81,7 +91,8 @@ __device__ __forceinline__ void rope32(float *v, int dim0, int t, int y, int x,
 
 __global__ void __launch_bounds__(kThreads, 1)
     project_kernel(const __grid_constant__ ProjectParams p, const __grid_constant__ CUtensorMap tx,
-                   const __grid_constant__ CUtensorMap tw) {
+                   const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tq,
+                   const __grid_constant__ CUtensorMap tkv) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -118,6 +129,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tx);
       tma_prefetch_desc(&tw);
+      tma_prefetch_desc(&tq);
+      tma_prefetch_desc(&tkv);
       int issued = 0;
       for (int kb = 0; kb < n_kb; ++kb) {
         const int s = kb % kStages;
@@ -162,12 +175,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue --
+    // Warpgroup h drains page h of the tile; warp w holds rows 32 (w % 4) ..
+    // +31 (TMEM lanes), thread = one token row. The 256 features of the tile
+    // are two heads (head0, head0 + 1) of one section (q, k or v) with the
+    // same rotary angles per dimension, so each 32-dimension chunk of both
+    // heads is rotated with one set of (cos, sin) loads. Rounded bf16 rows are
+    // staged in the drained operand ring (128-byte swizzled, one 16 KB half
+    // per 64 dimensions) and every warp writes its 32 rows with TMA stores:
+    // q_rot through the activation map (rows past C clipped), K/V straight
+    // into the page rows (rows past C are zeros).
     const int h = warp >> 2;                             // page of the tile
     const int page = 2 * mt + h;                         // page of the chunk
-    const int r = (warp & 3) * 32 + lane;                // token row in the page == TMEM lane
+    const int wr = (warp & 3) * 32;                      // first row of this warp
+    const int r = wr + lane;                             // token row in the page == TMEM lane
     const int n = page * kPage + r;                      // token inside the chunk
     const bool valid = n < p.C;
-    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t lane_addr = static_cast<uint32_t>(wr) << 16;
     const bool ok = __all_sync(0xffffffffu, wait_bar(ctx, kAccFull, 0));
     if (ok && page < p.npc) {
       tc_fence_after();
@@ -181,48 +204,101 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int pos = __ldg(p.table + kTabSlotPos + slot);
       int phys = pos < 0 ? -1 : __ldg(p.table + kTabPages + pos * p.npc + page);
       if (phys >= p.num_pages) phys = -1;
-      const size_t page_elems = static_cast<size_t>(2) * p.Hh * p.P * p.d;
-#pragma unroll 1
-      for (int c = 0; c < kGN / 32; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(tmem + lane_addr + h * kGN + c * 32, raw);
-        tmem_ld_wait();
-        reg_fence32(raw);
-        const int f0 = nt * kGN + c * 32;                // first output feature of the piece
-        const int sec = f0 / p.hidden;                   // 0 q, 1 k, 2 v
-        const int within = f0 - sec * p.hidden;
-        const int head = within / p.d;
-        const int dim0 = within - head * p.d;
-        float v[32];
+      const int f0 = nt * kGN;                           // first output feature of the tile
+      const int sec = f0 / p.hidden;                     // 0 q, 1 k, 2 v
+      const int head0 = (f0 - sec * p.hidden) / p.d;     // heads head0, head0 + 1
+      const bool rot = sec < 2 && p.rope && valid;
+      uint8_t *stage = smem + h * 2 * kHeadStage;        // [head slot][64-dim half][128 rows][128 B]
+      const int h0 = p.split0 >> 1, h1 = p.split1 >> 1, h2 = p.split2 >> 1;
+      const bool kv_ok = sec > 0 && phys >= 0;
+      if (lane == 0 && sec > 0 && phys < 0) record_status(p.status, WF_ERR_BAD_PAGE);
+      // (cos, sin) of the 16 pairs of dimensions 32 c .. 32 c + 31; the band of
+      // a pair is picked by selects, and all 16 loads issue before any use.
+      auto load_cs = [&](int c, float2 (&cs)[16]) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
-        if (sec < 2 && p.rope && valid) rope32(v, dim0, tpos, ypos, xpos, p);
+        for (int i = 0; i < 16; ++i) {
+          const int pr = c * 16 + i;
+          const float2 *src = pr < h0        ? p.rope_t + tpos * h0 + pr
+                              : pr < h0 + h1 ? p.rope_h + ypos * h1 + (pr - h0)
+                                             : p.rope_w + xpos * h2 + (pr - h0 - h1);
+          cs[i] = __ldg(src);
+        }
+      };
+      // Step s drains dimensions 32 c .. 32 c + 31 (c = s / 2) of head slot
+      // hs = s % 2 while the TMEM load of step s + 1 and, on even steps, the
+      // (cos, sin) of the next chunk are in flight. The 64-dimension half kt
+      // of both heads is complete after steps 3 and 7; its TMA stores are
+      // issued at once, so the first half's stores overlap the second half.
+      uint32_t cur[32], nxt[32];
+      float2 cs[16], csn[16];
+      tmem_ld32(tmem + lane_addr + h * kGN, cur);
+      if (rot) load_cs(0, cs);
+      tmem_ld_wait();
+      reg_fence32(cur);
+#pragma unroll
+      for (int st = 0; st < 8; ++st) {
+        const int c = st >> 1, hs = st & 1, kt = c >> 1;
+        if (st < 7) {
+          const int cn = (st + 1) >> 1, hn = (st + 1) & 1;
+          tmem_ld32(tmem + lane_addr + h * kGN + hn * 128 + cn * 32, nxt);
+        }
+        if (rot && hs == 0 && c < 3) load_cs(c + 1, csn);
+        if (rot) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a = __uint_as_float(cur[2 * i]), b = __uint_as_float(cur[2 * i + 1]);
+            cur[2 * i] = __float_as_uint(a * cs[i].x - b * cs[i].y);
+            cur[2 * i + 1] = __float_as_uint(a * cs[i].y + b * cs[i].x);
+          }
+        }
         uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = valid ? pack_bf16(v[2 * i], v[2 * i + 1]) : 0u;
-        // Lanes decide independently whether and where to store; the warp
-        // stays converged for the next tcgen05.ld.
-        uint4 *dst = nullptr;
-        if (sec == 0) {
-          if (valid)
-            dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.q_rot) +
-                                            ((static_cast<size_t>(slot) * p.C + n) * p.Hh + head) *
-                                                p.d + dim0);
-        } else if (phys < 0) {
-          record_status(p.status, WF_ERR_BAD_PAGE);
-        } else {
-          dst = reinterpret_cast<uint4 *>(
-              reinterpret_cast<__nv_bfloat16 *>(p.pages) + phys * page_elems +
-              ((static_cast<size_t>(sec - 1) * p.Hh + head) * p.P + r) * p.d + dim0);
-          if (sec == 1 && head == 0 && dim0 == 0 && r == 0) p.tags[phys] = p.live.tag[li];
-        }
-        if (dst != nullptr) {
+        for (int i = 0; i < 16; ++i)
+          w[i] = valid ? pack_bf16(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])) : 0u;
+        uint8_t *half = stage + hs * kHeadStage + kt * kHalfStage + r * 128;
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        for (int i = 0; i < 4; ++i) {
+          const int chunk = (c & 1) * 4 + i;             // 16-byte chunk of the 128-byte row
+          const uint32_t addr = smem_u32(half + ((chunk ^ (r & 7)) << 4));
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[4 * i]),
+                       "r"(w[4 * i + 1]), "r"(w[4 * i + 2]), "r"(w[4 * i + 3])
+                       : "memory");
         }
-        __syncwarp();
+        if (st == 3 || st == 7) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint8_t *src = stage + hh * kHeadStage + kt * kHalfStage + wr * 128;
+              if (sec == 0) {
+                if (page * kPage + wr < p.C)            // boxes wholly past C are skipped
+                  tma_store_4d(&tq, src, kt * 64, head0 + hh, page * kPage + wr, slot);
+              } else if (kv_ok) {
+                const int64_t row = p.layer_row0 +
+                    ((static_cast<int64_t>(phys) * 2 + (sec - 1)) * p.Hh + head0 + hh) * p.P + wr;
+                tma_store_2d(&tkv, src, kt * 64, static_cast<int>(row));
+              }
+            }
+            tma_store_commit();
+          }
+        }
+        if (st < 7) {
+          tmem_ld_wait();
+          reg_fence32(nxt);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) cur[i] = nxt[i];
+        }
+        if (rot && hs == 1 && c < 3) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) cs[i] = csn[i];
+        }
       }
+      if (lane == 0) {
+        tma_store_wait_all();                            // the staging smem stays live until read
+        if (sec == 1 && head0 == 0 && wr == 0 && kv_ok) p.tags[phys] = p.live.tag[li];
+      }
+      __syncwarp();
     }
   }
 
@@ -237,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_project_bf16(const ProjectParams &p, const void *tmap_x, const void *tmap_w,
-                                cudaStream_t st) {
+                                const void *tmap_q, const void *tmap_kv, cudaStream_t st) {
   if (p.live.n == 0) return cudaSuccess;
   if (p.d != 128 || p.P != kPage || p.hidden % kGN != 0) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -246,7 +322,8 @@ cudaError_t launch_project_bf16(const ProjectParams &p, const void *tmap_x, cons
   const int64_t blocks = static_cast<int64_t>(p.live.n) * ((p.npc + 1) / 2) * (3 * p.hidden / kGN);
   if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
   project_kernel<<<static_cast<unsigned>(blocks), kThreads, kSmemBytes, st>>>(
-      p, *static_cast<const CUtensorMap *>(tmap_x), *static_cast<const CUtensorMap *>(tmap_w));
+      p, *static_cast<const CUtensorMap *>(tmap_x), *static_cast<const CUtensorMap *>(tmap_w),
+      *static_cast<const CUtensorMap *>(tmap_q), *static_cast<const CUtensorMap *>(tmap_kv));
   return cudaGetLastError();
 }
 

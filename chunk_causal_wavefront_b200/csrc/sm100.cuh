@@ -90,6 +90,13 @@ __device__ __forceinline__ void tma_store_4d(const void *desc, const void *src, 
       : "memory");
 }
 
+__device__ __forceinline__ void tma_store_2d(const void *desc, const void *src, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(desc),
+      "r"(smem_u32(src)), "r"(x), "r"(y)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_store_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

@@ -78,6 +78,7 @@ struct ProjectParams {
   const float2 *rope_t, *rope_h, *rope_w;
   int32_t S1, C, Hh, d, P, npc, num_pages, hidden;
   int32_t rope, F, gh, gw, split0, split1, split2;
+  int64_t layer_row0;         // first pool row of this layer (pool store tensor map)
   LiveSlots live;
 };
 
@@ -100,9 +101,11 @@ cudaError_t launch_attention_bf16(const AttnParams &p, const void *tmap_q,
 cudaError_t launch_attention_fp8(const AttnParams &p, const void *tmap_q,
                                  const void *tmap_kv, const void *tmap_out, cudaStream_t st);
 // Fused QKV projection: tensor maps of x (3D: hidden x C x S+1, box 64 x 256 x 1)
-// and w_qkv (2D: hidden x 3*hidden, box 64 x 256).
+// and w_qkv (2D: hidden x 3*hidden, box 64 x 256) for the operands, and the two
+// store maps of the epilogue: q_rot (4D [S+1][C][heads][d], box 64 x 1 x 32 x 1)
+// and the pool's K/V rows (2D [rows][d], box 64 x 32), all 128-byte swizzled.
 cudaError_t launch_project_bf16(const ProjectParams &p, const void *tmap_x, const void *tmap_w,
-                                cudaStream_t st);
+                                const void *tmap_q, const void *tmap_kv, cudaStream_t st);
 cudaError_t launch_table_upload(int32_t *dst, const int32_t *src, int n_words,
                                 cudaStream_t st);
 cudaError_t launch_poke(int32_t *dst, int32_t value, cudaStream_t st);
