@@ -41,6 +41,25 @@ __device__ __forceinline__ bool wait_bar(const Ctx &c, int b, uint32_t parity) {
   }
 }
 
+// Bounded wait on a phase completed (in part) by the other CTA of a pair:
+// acquire at cluster scope.
+__device__ __forceinline__ bool wait_bar_cluster(const Ctx &c, int b, uint32_t parity) {
+  uint64_t *bar = c.bars + b;
+  if (sm100::mbar_try_wait_cluster(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (sm100::mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 127u) == 0) {
+      if (*c.abort) return false;
+      if (clock64() - t0 > kWaitLimit) {
+        *c.abort = 1;
+        record_status(c.status, WF_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
 // Time-bounded wait used while draining (ignores the abort flag).
 __device__ __forceinline__ void drain_wait(const Ctx &c, int b, uint32_t parity) {
   uint64_t *bar = c.bars + b;

@@ -558,11 +558,11 @@ wf_status wf_project_publish(wf_pool *p, int32_t layer, const void *x, const voi
                             static_cast<cuuint64_t>(c.num_stages + 1)};
   const cuuint64_t xs[2] = {static_cast<cuuint64_t>(hidden) * 2,
                             static_cast<cuuint64_t>(hidden) * 2 * c.chunk_tokens};
-  const cuuint32_t xb[3] = {64, 256, 1};
+  const cuuint32_t xb[3] = {64, 128, 1};   // one page per CTA of a pair
   if (!encode_bf16_map(&xmap, const_cast<void *>(x), 3, xd, xs, xb)) return WF_ERR_CUDA;
   const cuuint64_t wd[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(3 * hidden)};
   const cuuint64_t ws[1] = {static_cast<cuuint64_t>(hidden) * 2};
-  const cuuint32_t wb[2] = {64, 256};
+  const cuuint32_t wb[2] = {64, 128};      // half of a tile's features per CTA
   if (!encode_bf16_map(&wmap, const_cast<void *>(w_qkv), 2, wd, ws, wb)) return WF_ERR_CUDA;
   // Epilogue stores: q_rot [S+1][C][heads][d] and the pool's K/V rows, 32 rows per box.
   const cuuint64_t qd[4] = {static_cast<cuuint64_t>(c.head_dim), static_cast<cuuint64_t>(c.num_heads),
