@@ -22,7 +22,7 @@
 //   tiles fastest, so the x pages and all of w stay in L2). Accumulators are
 //   double-buffered in TMEM (columns [256 b, 256 b + 256)), so the epilogue of
 //   one tile overlaps the main loop of the next.
-//   warp 8 (one lane)  TMA producer of its CTA: a 4-stage ring of 32 KB stages
+//   warp 8 (one lane)  TMA producer of its CTA: a 6-stage ring of 32 KB stages
 //                      (128-byte swizzle); the loads of both CTAs count on the
 //                      leader's full barrier, and the leader's commits free the
 //                      stage in both CTAs.
@@ -54,15 +54,16 @@ constexpr int kPage = 128;                    // tokens per page (M per CTA)
 constexpr int kGN = 256;                      // output features per tile (N)
 constexpr int kHalfN = kGN / 2;               // features of w held by each CTA
 constexpr int kGK = 64;                       // hidden elements per k-block (128 bytes)
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr uint32_t kABytes = kPage * kGK * 2;     // 16 KB
 constexpr uint32_t kBBytes = kHalfN * kGK * 2;    // 16 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
-// Epilogue staging: per head slot, two 64-dimension halves of 128 rows x 128 B.
+// Epilogue staging: per head slot, one 64-dimension half of 128 rows x 128 B
+// at a time (each warp's 32 rows are its own; the second half waits until the
+// first half's TMA store has read them).
 constexpr uint32_t kHalfStage = kPage * 128;      // 16 KB
-constexpr uint32_t kHeadStage = 2 * kHalfStage;   // 32 KB
 constexpr uint32_t kOffStage = kStages * kStageBytes;
-constexpr uint32_t kOffBar = kOffStage + 2 * kHeadStage;
+constexpr uint32_t kOffBar = kOffStage + 2 * kHalfStage;
 constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
 constexpr int kProducerWarp = 8;
@@ -207,7 +208,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int wr = (warp & 3) * 32;                      // first row of this warp
     const int r = wr + lane;                             // token row in the page == TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(wr) << 16;
-    uint8_t *stage = smem + kOffStage + e * kHeadStage;  // [64-dim half][128 rows][128 B]
+    uint8_t *stage = smem + kOffStage + e * kHalfStage;  // [128 rows][128 B]
     const int h0 = p.split0 >> 1, h1 = p.split1 >> 1, h2 = p.split2 >> 1;
     int i = 0;
     for (int t = pair; t < total; t += npairs, ++i) {
@@ -259,7 +260,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          const uint8_t *src = stage + kt * kHalfStage + wr * 128;
+          const uint8_t *src = stage + wr * 128;
           if (sec == 0) {
             if (page * kPage + wr < p.C)                 // boxes wholly past C are skipped
               tma_store_4d(&tq, src, kt * 64, head, page * kPage + wr, slot);
@@ -295,12 +296,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             cur[2 * q + 1] = __float_as_uint(a * cs[q].y + bb * cs[q].x);
           }
         }
+        if (live_page && c == 2) {
+          // The first half's TMA store has read this warp's staging rows.
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          __syncwarp();
+        }
         if (live_page) {
           uint32_t w[16];
 #pragma unroll
           for (int q = 0; q < 16; ++q)
             w[q] = valid ? pack_bf16(__uint_as_float(cur[2 * q]), __uint_as_float(cur[2 * q + 1])) : 0u;
-          uint8_t *row = stage + (c >> 1) * kHalfStage + r * 128;
+          uint8_t *row = stage + r * 128;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int chunk = (c & 1) * 4 + q;           // 16-byte chunk of the 128-byte row

@@ -1,6 +1,7 @@
-// Thin inline-PTX wrappers for the sm_100a features the attention kernel uses:
+// Thin inline-PTX wrappers for the sm_100a features the kernels use:
 // mbarriers, TMA tile loads, and the 5th-generation tensor core (tcgen05) with
-// its tensor memory (TMEM). Only non-multicast forms are used.
+// its tensor memory (TMEM). TMA loads use no multicast; only the CTA-pair commit
+// multicasts its mbarrier arrival to both CTAs of the pair.
 #pragma once
 
 #include <cstdint>
