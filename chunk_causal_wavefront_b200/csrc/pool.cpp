@@ -438,7 +438,8 @@ wf_status wf_publish_kv(wf_pool *p, int32_t layer, const void *q, const void *k,
   }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (c.dtype == WF_DTYPE_FP8_E4M3) {
+  const bool tiled = c.head_dim == 128 && c.page_tokens == 128;
+  if (c.dtype == WF_DTYPE_FP8_E4M3 || (c.dtype == WF_DTYPE_BF16 && tiled)) {
     // [S+1][C][heads][d] bf16; one box is a 128-row tile of one head.
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(c.head_dim),
                                 static_cast<cuuint64_t>(c.num_heads),
@@ -452,7 +453,21 @@ wf_status wf_publish_kv(wf_pool *p, int32_t layer, const void *q, const void *k,
         !encode_plain_bf16_map(&mk, const_cast<void *>(k), 4, dims, strides, box) ||
         !encode_plain_bf16_map(&mv, const_cast<void *>(v), 4, dims, strides, box))
       return WF_ERR_CUDA;
-    e = launch_publish_fp8(pp, &mq, &mk, &mv, cs);
+    if (c.dtype == WF_DTYPE_FP8_E4M3) {
+      e = launch_publish_fp8(pp, &mq, &mk, &mv, cs);
+    } else {
+      // q_rot as the inputs; the layer's pages as [pages x 2 x heads x P rows][d].
+      const cuuint64_t pdims[2] = {static_cast<cuuint64_t>(c.head_dim),
+                                   static_cast<cuuint64_t>(p->g.num_pages) * 2 * c.num_heads *
+                                       c.page_tokens};
+      const cuuint64_t pstrides[1] = {row};
+      const cuuint32_t pbox[2] = {128, 128};
+      CUtensorMap mqr, mpg;
+      if (!encode_plain_bf16_map(&mqr, q_rot, 4, dims, strides, box) ||
+          !encode_plain_bf16_map(&mpg, pp.pages, 2, pdims, pstrides, pbox))
+        return WF_ERR_CUDA;
+      e = launch_publish_bf16_tma(pp, &mq, &mk, &mv, &mqr, &mpg, cs);
+    }
   } else {
     e = c.dtype == WF_DTYPE_BF16 ? launch_publish_bf16(pp, cs) : launch_publish_f32(pp, cs);
   }

@@ -106,6 +106,13 @@ __device__ __forceinline__ void tma_store_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// Wait until every committed bulk store has finished reading shared memory
+// (the source buffers may be overwritten; the global writes may still be in
+// flight).
+__device__ __forceinline__ void tma_store_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // Make generic-proxy shared-memory writes visible to the async proxy
 // (tensor core and TMA reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
