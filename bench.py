@@ -624,7 +624,10 @@ def main():
                           "pct_peak_burst": 100 * att_tflops / (ratio * peaks["bf16_tflops"]),
                           "pct_peak_sustained": 100 * att_tflops / (ratio * peak),
                           "flops_per_launch": res["flops"]},
-            "publish": ({"ms_per_launch": res["pub_ms"], "gbs": pub_gbs,
+            "publish": ({"kernel": ("publish_fp8_kernel" if f8 else
+                                    "publish_tma_kernel" if cfg.head_dim == 128 and cfg.page_tokens == 128
+                                    else "publish_kernel"),
+                         "ms_per_launch": res["pub_ms"], "gbs": pub_gbs,
                          "pct_hbm": 100 * pub_gbs / peaks["hbm_gbs"],
                          "bytes_per_launch": res["pbytes"]} if not args.fused else
                         {"kernel": "project_kernel (QKV GEMM + RoPE + paged publication)",
