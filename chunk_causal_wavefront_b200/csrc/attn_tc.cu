@@ -96,7 +96,7 @@ struct Fmt {
   static constexpr uint32_t kOffBar = kF8 ? kOffStage + 2 * 32768 : kOffStage;
   static constexpr float kLazy = kF8 ? 4.0f : 8.0f;             // rescale threshold (log2)
   static constexpr int kPShift = 4;                             // E4M3 headroom of P'
-  static constexpr int kNumBars = 16;
+  static constexpr int kNumBars = 24;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // TMEM base, abort, 12 ints
   static constexpr uint32_t kOffPages = kOffMisc + 64;
   static constexpr uint32_t kOffExps = kOffPages + kPageCache * 4;   // int16 ek, ev (FP8)
@@ -106,7 +106,8 @@ struct Fmt {
 constexpr int kNumBars = Fmt<false>::kNumBars;
 enum Bar {
   kQFull = 0, kKFull0 = 1, kKEmpty0 = 3, kVFull0 = 5, kVEmpty0 = 7,
-  kSFull0 = 9, kPReady0 = 11, kPVDone0 = 13, kDrain = 15
+  kSFull0 = 9, kPReady0 = 11, kPVDone0 = 13, kDrain = 15,
+  kTurn0 = 16, kTurn1 = 20   // E4M3: exponential-phase turns, one per sub-partition and tile
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -448,6 +449,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P = 2^(s * c_j - m [+ dv]) on the MUFU unit, the scale-subtract and
       // the row sums in packed f32x2 arithmetic; rounded to the operand format
       // and streamed back into the first columns of S_q, 32 keys at a time.
+      // E4M3: the two tiles' softmax warps of a sub-partition take turns on the
+      // exponentials (tile 0 first), so that each runs them with the MUFU unit
+      // to itself; the turn is handed on after three quarters of the row. With
+      // the FP8 MMAs' shorter P*V + S the two phases would otherwise overlap
+      // (bf16 tiles stay apart by themselves, and a turn only delays them).
+      if (kF8 && has_q1 && (q == 1 || j > 0)) {
+        ok = __all_sync(0xffffffffu, wait_bar(ctx, (q == 0 ? kTurn0 : kTurn1) + (warp & 3),
+                                              q == 0 ? ((j - 1) & 1) : (j & 1)));
+        if (!ok) break;
+      }
       const uint64_t sc2 = f2(c_j, c_j), nm2 = f2(dv - m_use, dv - m_use);
       uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -467,6 +478,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             else half = pr;
           }
           tmem_st8(tS + cc * 8, pw);
+          if (cc == 2 && has_q1 && lane == 0)
+            mbar_arrive(bars + (q == 0 ? kTurn1 : kTurn0) + (warp & 3));
         } else {
           uint32_t pw[16];
 #pragma unroll
