@@ -22,6 +22,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -100,8 +101,12 @@ def read_peaks():
 
 
 def source_sha(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of a kernel source's code: line comments and blank lines are left
+    out, so that a comment edit does not void the recorded counters."""
+    with open(path, encoding="utf-8") as f:
+        lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in f]
+    code = "\n".join(ln for ln in lines if ln.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def read_traffic(kernel_file, variant=None):

@@ -27,7 +27,11 @@
 //                      the running max grows by more than a threshold (lazy
 //                      rescaling: the exponentials stay below 2^threshold
 //                      otherwise), the only time softmax waits for the previous
-//                      P*V. The epilogue divides by the row sum, stages bf16
+//                      P*V. Only the row max and the exponentials sit between
+//                      S ready and P ready: the row sum and the correction
+//                      factor are updated after P is handed over, and the
+//                      last-page test is taken before the wait for S. The
+//                      epilogue divides by the row sum, stages bf16
 //                      rows in shared memory and each warp writes its 32 rows
 //                      with a TMA store that clips rows past C.
 // Operand formats:
@@ -42,7 +46,11 @@
 //         units of 2^(ev_max - 4) and the row sum adds P'_j * 2^(ev_max + 4 - ev_j).
 //         The lazy threshold is 2^4, so P' <= 2^8 stays inside E4M3's range
 //         (448) while small probabilities keep 4 more binades above its
-//         subnormal range.
+//         subnormal range. With the MMAs at twice the bf16 rate the two tiles'
+//         exponential phases would overlap on the MUFU unit, so the softmax
+//         warps of a sub-partition take turns on them (one mbarrier per
+//         sub-partition and tile; the turn passes after three quarters of the
+//         row).
 // Every wait is bounded: on timeout the CTA records WF_ERR_TIMEOUT, the other
 // roles see the abort flag, in-flight copies and MMAs are drained and TMEM is
 // freed before the CTA exits.
