@@ -440,14 +440,15 @@ wf_status wf_publish_kv(wf_pool *p, int32_t layer, const void *q, const void *k,
   cudaError_t e;
   const bool tiled = c.head_dim == 128 && c.page_tokens == 128;
   if (c.dtype == WF_DTYPE_FP8_E4M3 || (c.dtype == WF_DTYPE_BF16 && tiled)) {
-    // [S+1][C][heads][d] bf16; one box is a 128-row tile of one head.
+    // [S+1][C][heads][d] bf16; one box is a 128-row (FP8 publish) or 64-row
+    // (bf16 publish) tile of one head.
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(c.head_dim),
                                 static_cast<cuuint64_t>(c.num_heads),
                                 static_cast<cuuint64_t>(c.chunk_tokens),
                                 static_cast<cuuint64_t>(c.num_stages + 1)};
     const cuuint64_t row = static_cast<cuuint64_t>(c.head_dim) * 2;
     const cuuint64_t strides[3] = {row, row * c.num_heads, row * c.num_heads * c.chunk_tokens};
-    const cuuint32_t box[4] = {128, 1, 128, 1};
+    const cuuint32_t box[4] = {128, 1, c.dtype == WF_DTYPE_FP8_E4M3 ? 128u : 64u, 1};
     CUtensorMap mq, mk, mv;
     if (!encode_plain_bf16_map(&mq, const_cast<void *>(q), 4, dims, strides, box) ||
         !encode_plain_bf16_map(&mk, const_cast<void *>(k), 4, dims, strides, box) ||
@@ -456,12 +457,13 @@ wf_status wf_publish_kv(wf_pool *p, int32_t layer, const void *q, const void *k,
     if (c.dtype == WF_DTYPE_FP8_E4M3) {
       e = launch_publish_fp8(pp, &mq, &mk, &mv, cs);
     } else {
-      // q_rot as the inputs; the layer's pages as [pages x 2 x heads x P rows][d].
+      // q_rot as the inputs; the layer's pages as [pages x 2 x heads x P rows][d],
+      // box 64 rows.
       const cuuint64_t pdims[2] = {static_cast<cuuint64_t>(c.head_dim),
                                    static_cast<cuuint64_t>(p->g.num_pages) * 2 * c.num_heads *
                                        c.page_tokens};
       const cuuint64_t pstrides[1] = {row};
-      const cuuint32_t pbox[2] = {128, 128};
+      const cuuint32_t pbox[2] = {128, 64};
       CUtensorMap mqr, mpg;
       if (!encode_plain_bf16_map(&mqr, q_rot, 4, dims, strides, box) ||
           !encode_plain_bf16_map(&mpg, pp.pages, 2, pdims, pstrides, pbox))

@@ -6,15 +6,17 @@
 // paged delivery writes them directly into ordered attention slots, followed
 // by a ready signal (here a per-page tag).
 //
-// Work unit: one (live slot, page j, head) block, i.e. 128 token rows x 128
-// dims of q, k and v (96 KB of bf16 in, 96 KB out). The kernel is persistent,
-// one CTA per SM walking the blocks blockIdx.x, blockIdx.x + gridDim.x, ...
-// through a two-stage shared-memory ring:
-//   * a TMA warp loads a block's q, k and v tiles (box 128 dims x 1 head x 128
-//     rows, rows past C zero-filled), and once the block is rotated stores the
+// Work unit: one half of a (live slot, page j, head) block, i.e. 64 token rows
+// x 128 dims of q, k and v (48 KB of bf16 in, 48 KB out). The kernel is
+// persistent, one CTA per SM walking the units blockIdx.x, blockIdx.x +
+// gridDim.x, ... through a four-stage shared-memory ring (half-page units in
+// four stages timed 3 % faster than whole pages in two, quarter pages slower):
+//   * a TMA warp loads a unit's q, k and v tiles (box 128 dims x 1 head x 64
+//     rows, rows past C zero-filled), and once the unit is rotated stores the
 //     q_rot tile (rows past C clipped by the tensor map) and the K and V tiles
-//     into the block's page (a 2D map over the layer's pool rows); it refills
-//     the stage with the next-but-one block as soon as the stores have read it;
+//     into the unit's half of the page (a 2D map over the layer's pool rows);
+//     it refills the stage with the unit four steps ahead as soon as the
+//     stores have read it;
 //   * 512 threads rotate q and k in place in shared memory, 16 threads per row
 //     (16 bytes = 4 rotary pairs each), in fp32 with one rounding to bf16;
 //     rows past C stay +0 (rotating them could turn +0 into -0); V is stored
@@ -32,33 +34,38 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kRows = 128;                             // rows per block (one page)
+constexpr int kRows = 64;                              // token rows per unit (half a page)
+constexpr int kPage = 128;                             // token rows per page
+constexpr int kSplit = kPage / kRows;                  // units per (page, head)
 constexpr int kComputeThreads = 512;
 constexpr int kComputeWarps = kComputeThreads / 32;    // 16
 constexpr int kThreads = kComputeThreads + 32;         // + the TMA warp
 constexpr int kTPR = 16;                               // threads per row
 constexpr int kRowsPerPass = kComputeThreads / kTPR;   // 32
-constexpr int kPasses = kRows / kRowsPerPass;          // 4
-constexpr uint32_t kTileBytes = kRows * 128 * 2;       // one bf16 tile, 32 KB
+constexpr int kPasses = kRows / kRowsPerPass;          // 2
+constexpr uint32_t kTileBytes = kRows * 128 * 2;       // one bf16 tile, 16 KB
 constexpr uint32_t kStageBytes = 3 * kTileBytes;       // q, k, v
-constexpr int kStages = 2;
-constexpr uint32_t kOffBars = kStages * kStageBytes;   // full[2], rotated[2]
-constexpr uint32_t kOffMisc = kOffBars + 64;           // abort flag
+constexpr int kStages = 4;
+constexpr uint32_t kOffBars = kStages * kStageBytes;   // full[kStages], rotated[kStages]
+constexpr uint32_t kOffMisc = kOffBars + 2 * kStages * 8;  // abort flag
 constexpr uint32_t kOffPos = kOffMisc + 64;            // [stage][row][4] rotary offsets
 constexpr uint32_t kSmemBytes = kOffPos + kStages * kRows * 4 * 4 + 1024;
-enum { kFull0 = 0, kRotated0 = 2 };
+enum { kFull0 = 0, kRotated0 = kStages };
 
-struct Block {
-  int li, j, h;
+struct Unit {
+  int li, j, h, row0, part;
 };
 
-__device__ __forceinline__ Block decode(int b, const PublishParams &p) {
-  Block k;
-  const int per_slot = p.npc * p.Hh;
+__device__ __forceinline__ Unit decode(int b, const PublishParams &p) {
+  Unit k;
+  const int per_slot = p.npc * kSplit * p.Hh;
   k.li = b / per_slot;
   const int rem = b - k.li * per_slot;
-  k.j = rem / p.Hh;
-  k.h = rem - k.j * p.Hh;
+  const int jp = rem / p.Hh;
+  k.h = rem - jp * p.Hh;
+  k.j = jp / kSplit;
+  k.part = jp - k.j * kSplit;
+  k.row0 = k.j * kPage + k.part * kRows;
   return k;
 }
 
@@ -69,16 +76,16 @@ __device__ __forceinline__ int block_page(const PublishParams &p, int slot, int 
   return (phys < 0 || phys >= p.num_pages) ? -1 : phys;
 }
 
-// The three TMA tile loads of block b into stage buffer `buf`.
-__device__ __forceinline__ void load_block(int b, uint8_t *buf, uint64_t *bar,
+// The three TMA tile loads of unit b into stage buffer `buf`.
+__device__ __forceinline__ void load_unit(int b, uint8_t *buf, uint64_t *bar,
                                            const PublishParams &p, const CUtensorMap *tq,
                                            const CUtensorMap *tk, const CUtensorMap *tv) {
-  const Block k = decode(b, p);
+  const Unit k = decode(b, p);
   const int slot = p.live.slot[k.li];
   mbar_arrive_expect_tx(bar, kStageBytes);
-  tma_load_4d(buf, tq, bar, 0, k.h, k.j * kRows, slot);
-  tma_load_4d(buf + kTileBytes, tk, bar, 0, k.h, k.j * kRows, slot);
-  tma_load_4d(buf + 2 * kTileBytes, tv, bar, 0, k.h, k.j * kRows, slot);
+  tma_load_4d(buf, tq, bar, 0, k.h, k.row0, slot);
+  tma_load_4d(buf + kTileBytes, tk, bar, 0, k.h, k.row0, slot);
+  tma_load_4d(buf + 2 * kTileBytes, tv, bar, 0, k.h, k.row0, slot);
 }
 
 // OR of a predicate over the 512 compute threads (named barrier 1), the same
@@ -120,16 +127,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc);
   int32_t *pos_all = reinterpret_cast<int32_t *>(smem + kOffPos);
-  const int nblk = p.live.n * p.npc * p.Hh;
+  const int nblk = p.live.n * p.npc * kSplit * p.Hh;
   const int G = gridDim.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Ctx ctx{bars, abort_flag, p.status};
 
   if (threadIdx.x == 0) {
-    mbar_init(bars + kFull0, 1);
-    mbar_init(bars + kFull0 + 1, 1);
-    mbar_init(bars + kRotated0, kComputeWarps);
-    mbar_init(bars + kRotated0 + 1, kComputeWarps);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bars + kFull0 + s, 1);
+      mbar_init(bars + kRotated0 + s, kComputeWarps);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -143,37 +150,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tv);
       tma_prefetch_desc(&tqr);
       tma_prefetch_desc(&tpg);
-      int issued[kStages] = {0, 0};
+      int issued[kStages] = {};
       for (int s = 0; s < kStages; ++s) {
         const int b = blockIdx.x + s * G;
         if (b < nblk) {
-          load_block(b, smem + s * kStageBytes, bars + kFull0 + s, p, &tq, &tk, &tv);
+          load_unit(b, smem + s * kStageBytes, bars + kFull0 + s, p, &tq, &tk, &tv);
           ++issued[s];
         }
       }
       for (int i = 0;; ++i) {
         const int b = blockIdx.x + i * G;
         if (b >= nblk) break;
-        const int s = i & 1;
-        if (!wait_bar(ctx, kRotated0 + s, (i >> 1) & 1)) break;
-        const Block blk = decode(b, p);
+        const int s = i % kStages;
+        if (!wait_bar(ctx, kRotated0 + s, (i / kStages) & 1)) break;
+        const Unit blk = decode(b, p);
         const int slot = p.live.slot[blk.li];
         const int phys = block_page(p, slot, blk.j);
         const uint8_t *buf = smem + s * kStageBytes;
-        tma_store_4d(&tqr, buf, 0, blk.h, blk.j * kRows, slot);
+        tma_store_4d(&tqr, buf, 0, blk.h, blk.row0, slot);
         if (phys >= 0) {
-          const int rowk = (phys * 2 * p.Hh + blk.h) * kRows;
+          const int rowk = (phys * 2 * p.Hh + blk.h) * kPage + blk.part * kRows;
           tma_store_2d(&tpg, buf + kTileBytes, 0, rowk);
-          tma_store_2d(&tpg, buf + 2 * kTileBytes, 0, rowk + p.Hh * kRows);
-          if (blk.h == 0) p.tags[phys] = p.live.tag[blk.li];
+          tma_store_2d(&tpg, buf + 2 * kTileBytes, 0, rowk + p.Hh * kPage);
+          if (blk.h == 0 && blk.part == 0) p.tags[phys] = p.live.tag[blk.li];
         } else {
           record_status(p.status, WF_ERR_BAD_PAGE);
         }
         tma_store_commit();
-        // Refill the stage with the next-but-one block once the stores have read it.
-        if (b + 2 * G < nblk) {
+        // Refill the stage with the unit kStages ahead once the stores have read it.
+        if (b + kStages * G < nblk) {
           tma_store_wait_read_all();
-          load_block(b + 2 * G, smem + s * kStageBytes, bars + kFull0 + s, p, &tq, &tk, &tv);
+          load_unit(b + kStages * G, smem + s * kStageBytes, bars + kFull0 + s, p, &tq, &tk, &tv);
           ++issued[s];
         }
       }
@@ -209,14 +216,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = 0;; ++i) {
     const int b = blockIdx.x + i * G;
     if (b >= nblk) break;
-    const int s = i & 1;
-    const Block blk = decode(b, p);
-    const int li = blk.li, j = blk.j;
+    const int s = i % kStages;
+    const Unit blk = decode(b, p);
+    const int li = blk.li;
     int32_t *pos = pos_all + s * kRows * 4;
-    // Rotary positions of the block's rows (absolute: frame F * chunk + n / (gh gw)).
+    // Rotary positions of the unit's rows (absolute: frame F * chunk + n / (gh gw)).
     // The stage's previous readers finished before the last barrier.
     if (p.rope && threadIdx.x < kRows) {
-      int n = j * kRows + threadIdx.x;
+      int n = blk.row0 + threadIdx.x;
       if (n >= p.C) n = 0;
       const int hw = p.gh * p.gw, f = n / hw, yx = n - f * hw, y = yx / p.gw;
       pos[4 * threadIdx.x] = (p.F * p.live.chunk[li] + f) * h0;
@@ -224,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       pos[4 * threadIdx.x + 2] = (yx - y * p.gw) * h2;
     }
     // The n-th use of a stage waits for its n-th fill: parity (i / 2) & 1.
-    const bool ok = __all_sync(0xffffffffu, wait_bar(ctx, kFull0 + s, (i >> 1) & 1));
+    const bool ok = __all_sync(0xffffffffu, wait_bar(ctx, kFull0 + s, (i / kStages) & 1));
     if (compute_any(!ok)) break;                  // also publishes pos[]
 
     if (p.rope) {
@@ -232,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int ps = 0; ps < kPasses; ++ps) {
         const int r = r0 + ps * kRowsPerPass;
-        if (j * kRows + r >= p.C) continue;       // zero rows past C stay +0
+        if (blk.row0 + r >= p.C) continue;       // zero rows past C stay +0
         const uint32_t off = r * 256 + cv * 16;
         uint4 *qa = reinterpret_cast<uint4 *>(buf + off);
         uint4 *ka = reinterpret_cast<uint4 *>(buf + kTileBytes + off);
@@ -259,8 +266,8 @@ cudaError_t launch_publish_bf16_tma(const PublishParams &p, const void *tmap_q, 
                                     const void *tmap_v, const void *tmap_qrot,
                                     const void *tmap_pages, cudaStream_t st) {
   if (p.live.n == 0) return cudaSuccess;
-  if (p.d != 128 || p.P != kRows) return cudaErrorInvalidValue;
-  const int64_t nblk = static_cast<int64_t>(p.live.n) * p.npc * p.Hh;
+  if (p.d != 128 || p.P != kPage) return cudaErrorInvalidValue;
+  const int64_t nblk = static_cast<int64_t>(p.live.n) * p.npc * kSplit * p.Hh;
   if (nblk > 0x7fffffff) return cudaErrorInvalidValue;
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);

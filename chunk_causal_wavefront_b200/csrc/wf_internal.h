@@ -89,9 +89,10 @@ cudaError_t launch_publish_f32(const PublishParams &p, cudaStream_t st);
 // [S+1][C][heads][d] bf16 with a box of 128 dims x 1 head x 128 rows.
 cudaError_t launch_publish_fp8(const PublishParams &p, const void *tmap_q, const void *tmap_k,
                                const void *tmap_v, cudaStream_t st);
-// The bf16 publish for d = 128 and 128-token pages takes the same maps of q, k
-// and v, one of q_rot (same shape and box), and an unswizzled 2D map over the
-// layer's pool rows ([pages x 2 x heads x 128 rows][d] bf16, box 128 x 128).
+// The bf16 publish for d = 128 and 128-token pages takes unswizzled maps of q,
+// k, v and q_rot over [S+1][C][heads][d] bf16 with a box of 128 dims x 1 head x
+// 64 rows, and an unswizzled 2D map over the layer's pool rows
+// ([pages x 2 x heads x 128 rows][d] bf16, box 128 x 64).
 cudaError_t launch_publish_bf16_tma(const PublishParams &p, const void *tmap_q, const void *tmap_k,
                                     const void *tmap_v, const void *tmap_qrot,
                                     const void *tmap_pages, cudaStream_t st);
