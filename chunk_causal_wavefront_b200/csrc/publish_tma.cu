@@ -48,8 +48,7 @@ constexpr uint32_t kStageBytes = 3 * kTileBytes;       // q, k, v
 constexpr int kStages = 4;
 constexpr uint32_t kOffBars = kStages * kStageBytes;   // full[kStages], rotated[kStages]
 constexpr uint32_t kOffMisc = kOffBars + 2 * kStages * 8;  // abort flag
-constexpr uint32_t kOffPos = kOffMisc + 64;            // [stage][row][4] rotary offsets
-constexpr uint32_t kSmemBytes = kOffPos + kStages * kRows * 4 * 4 + 1024;
+constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
 enum { kFull0 = 0, kRotated0 = kStages };
 
 struct Unit {
@@ -126,7 +125,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc);
-  int32_t *pos_all = reinterpret_cast<int32_t *>(smem + kOffPos);
   const int nblk = p.live.n * p.npc * kSplit * p.Hh;
   const int G = gridDim.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -197,10 +195,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int cv = threadIdx.x & (kTPR - 1);        // 16-byte vector of the head row
   const int r0 = threadIdx.x / kTPR;              // first row of this thread
   // Rotary (cos, sin) entries of this thread's 4 pairs (pairs 4 cv .. 4 cv + 3):
-  // pair pr lies in band t, h or w (band index b); its entry for row r is
-  // rope_t[o + pos[4 r + b]], o the pair's offset from the t table (the three
-  // tables share the pool buffer) and pos the row's position in each band
-  // times that band's pair count. ctab[i] packs 4 o + b.
+  // pair pr lies in band t, h or w (band index b); its entry for a row is
+  // rope_t[o + q_b], o the pair's offset from the t table (the three tables
+  // share the pool buffer) and q_b the row's position in band b times that
+  // band's pair count. ctab[i] packs 4 o + b.
   const int h0 = p.split0 >> 1, h1 = p.split1 >> 1, h2 = p.split2 >> 1;
   int ctab[4] = {0, 0, 0, 0};
   if (p.rope) {
@@ -218,21 +216,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (b >= nblk) break;
     const int s = i % kStages;
     const Unit blk = decode(b, p);
-    const int li = blk.li;
-    int32_t *pos = pos_all + s * kRows * 4;
-    // Rotary positions of the unit's rows (absolute: frame F * chunk + n / (gh gw)).
-    // The stage's previous readers finished before the last barrier.
-    if (p.rope && threadIdx.x < kRows) {
-      int n = blk.row0 + threadIdx.x;
-      if (n >= p.C) n = 0;
-      const int hw = p.gh * p.gw, f = n / hw, yx = n - f * hw, y = yx / p.gw;
-      pos[4 * threadIdx.x] = (p.F * p.live.chunk[li] + f) * h0;
-      pos[4 * threadIdx.x + 1] = y * h1;
-      pos[4 * threadIdx.x + 2] = (yx - y * p.gw) * h2;
+    // The (cos, sin) entries of this thread's rows and pairs are loaded while
+    // the unit's tiles are still in flight. Rotary positions are absolute:
+    // frame F * chunk + n / (gh gw), row y, column x.
+    float2 cs[kPasses][4];
+    if (p.rope) {
+      const int hw = p.gh * p.gw, t0 = p.F * p.live.chunk[blk.li];
+#pragma unroll
+      for (int ps = 0; ps < kPasses; ++ps) {
+        int n = blk.row0 + r0 + ps * kRowsPerPass;
+        if (n >= p.C) n = 0;
+        const int f = n / hw, yx = n - f * hw, y = yx / p.gw;
+        const int pt = (t0 + f) * h0, py = y * h1, px = (yx - y * p.gw) * h2;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int band = ctab[c] & 3;
+          cs[ps][c] = __ldg(p.rope_t + (ctab[c] >> 2) + (band == 0 ? pt : band == 1 ? py : px));
+        }
+      }
     }
-    // The n-th use of a stage waits for its n-th fill: parity (i / 2) & 1.
+    // The n-th use of a stage waits for its n-th fill: parity (i / kStages) & 1.
     const bool ok = __all_sync(0xffffffffu, wait_bar(ctx, kFull0 + s, (i / kStages) & 1));
-    if (compute_any(!ok)) break;                  // also publishes pos[]
+    if (compute_any(!ok)) break;
 
     if (p.rope) {
       uint8_t *buf = smem + s * kStageBytes;
@@ -244,11 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint4 *qa = reinterpret_cast<uint4 *>(buf + off);
         uint4 *ka = reinterpret_cast<uint4 *>(buf + kTileBytes + off);
         uint4 qv = *qa, kv = *ka;
-        float2 cs[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) cs[c] = __ldg(p.rope_t + (ctab[c] >> 2) + pos[4 * r + (ctab[c] & 3)]);
-        rotate_vec(qv, cs);
-        rotate_vec(kv, cs);
+        rotate_vec(qv, cs[ps]);
+        rotate_vec(kv, cs[ps]);
         *qa = qv;
         *ka = kv;
       }
