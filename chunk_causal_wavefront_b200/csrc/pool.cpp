@@ -438,8 +438,7 @@ wf_status wf_publish_kv(wf_pool *p, int32_t layer, const void *q, const void *k,
   }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  const bool tiled = c.head_dim == 128 && c.page_tokens == 128;
-  if (c.dtype == WF_DTYPE_FP8_E4M3 || (c.dtype == WF_DTYPE_BF16 && tiled)) {
+  if (c.dtype == WF_DTYPE_FP8_E4M3 || c.dtype == WF_DTYPE_BF16) {   // d = P = 128 (validate)
     // [S+1][C][heads][d] bf16; one box is a 128-row (FP8 publish) or 64-row
     // (bf16 publish) tile of one head.
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(c.head_dim),
@@ -471,7 +470,7 @@ wf_status wf_publish_kv(wf_pool *p, int32_t layer, const void *q, const void *k,
       e = launch_publish_bf16_tma(pp, &mq, &mk, &mv, &mqr, &mpg, cs);
     }
   } else {
-    e = c.dtype == WF_DTYPE_BF16 ? launch_publish_bf16(pp, cs) : launch_publish_f32(pp, cs);
+    e = launch_publish_f32(pp, cs);
   }
   return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }

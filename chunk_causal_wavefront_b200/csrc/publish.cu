@@ -6,17 +6,18 @@
 // by a ready signal. Here the "slots" are the pages that the device page table
 // assigns to each live slot; the ready signal is a per-page tag.
 //
+// This kernel serves fp32 pools (any head_dim that is a multiple of 4 up to
+// 128, pages of up to 256 tokens); bf16 pools, whose head_dim and pages are
+// 128, publish through the TMA ring of publish_tma.cu.
+//
 // One launch covers every live slot of the round (grid row = slot). A thread
-// handles 16-byte vectors (8 bf16 or 4 fp32 values = 4 or 2 rotary pairs) of
-// (slot, token, head) rows, two per iteration: it loads q, k and v with
-// streaming 16-byte loads,
-// rotates q and k in fp32 with (cos, sin) tables computed on the host in fp64,
-// rounds once to the storage type and issues 16-byte stores to q_rot and to
-// the K and V pages. Consecutive threads cover consecutive 16-byte vectors of
-// the [C][heads][d] input rows, so loads are fully coalesced; a warp's page
-// stores cover two contiguous 256-byte head rows. HBM-bound: 3 reads + 3
-// writes of every element.
-#include <cuda_bf16.h>
+// handles 16-byte vectors (4 fp32 values = 2 rotary pairs) of (slot, token,
+// head) rows, two per iteration: it loads q, k and v with streaming 16-byte
+// loads, rotates q and k with (cos, sin) tables computed on the host in fp64,
+// and issues 16-byte stores to q_rot and to the K and V pages. Consecutive
+// threads cover consecutive 16-byte vectors of the [C][heads][d] input rows,
+// so loads are fully coalesced. HBM-bound: 3 reads + 3 writes of every
+// element.
 
 #include "wf_internal.h"
 
@@ -54,7 +55,6 @@ struct PublishDivs {
 };
 
 template <typename T> struct Vec;
-template <> struct Vec<__nv_bfloat16> { static constexpr int N = 8; };
 template <> struct Vec<float> { static constexpr int N = 4; };
 
 __device__ __forceinline__ uint4 ld_stream(const void *p) {
@@ -64,28 +64,11 @@ __device__ __forceinline__ uint4 ld_stream(const void *p) {
   return r;
 }
 
-__device__ __forceinline__ void unpack(const uint4 &u, float *f, __nv_bfloat16) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
 __device__ __forceinline__ void unpack(const uint4 &u, float *f, float) {
   f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
   f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
 }
 
-__device__ __forceinline__ uint4 pack(const float *f, __nv_bfloat16) {
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __nv_bfloat162 b = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);   // RNE
-    w[i] = *reinterpret_cast<uint32_t *>(&b);
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
-}
 __device__ __forceinline__ uint4 pack(const float *f, float) {
   return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
                     __float_as_uint(f[3]));
@@ -250,9 +233,6 @@ cudaError_t launch(const PublishParams &p, cudaStream_t st) {
 
 }  // namespace
 
-cudaError_t launch_publish_bf16(const PublishParams &p, cudaStream_t st) {
-  return launch<__nv_bfloat16>(p, st);
-}
 cudaError_t launch_publish_f32(const PublishParams &p, cudaStream_t st) {
   return launch<float>(p, st);
 }

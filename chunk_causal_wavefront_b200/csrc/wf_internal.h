@@ -83,7 +83,6 @@ struct ProjectParams {
 };
 
 // Launchers (return a cudaError_t from the launch).
-cudaError_t launch_publish_bf16(const PublishParams &p, cudaStream_t st);
 cudaError_t launch_publish_f32(const PublishParams &p, cudaStream_t st);
 // The FP8 publish takes unswizzled tensor maps of q, k and v over
 // [S+1][C][heads][d] bf16 with a box of 128 dims x 1 head x 128 rows.

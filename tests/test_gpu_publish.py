@@ -131,3 +131,23 @@ def test_publish_second_layer_independent():
     tags = ro.pool.tags_view().cpu().numpy()
     assert (tags[0] == 0).all() and (tags[1] == 0).all()
     ro.close()
+
+
+# The bf16 publish for 128-token pages moves half pages (64 rows) through TMA:
+# chunks that end exactly on or inside either half of a page, or below one
+# half, and one that fills its pages exactly.
+@pytest.mark.parametrize("C,gh,gw", [(40, 5, 8), (64, 8, 8), (100, 10, 10), (192, 12, 16),
+                                     (256, 16, 16)])
+def test_publish_half_page_boundaries(C, gh, gw):
+    cfg = wf_inputs.CONFIGS["wan13b_bf16"].replace(
+        num_stages=3, chunk_tokens=C, num_heads=3, history_chunks=1, frames_per_chunk=1,
+        grid_h=gh, grid_w=gw)
+    ro = Rollout(cfg, page_seed=C)
+    for _ in range(cfg.steady_round()):
+        ro.advance()
+    ro.publish(0)
+    torch.cuda.synchronize()
+    assert ro.pool.check_status() == 0
+    _check_round(ro)
+    ro.close()
+
