@@ -1,5 +1,6 @@
 // Early K/V publication into a bf16 pool with 128-token pages and d = 128:
-// rotary embedding + scatter of whole (page, head) tiles through TMA.
+// rotary embedding + scatter of (page, head) tiles, half a page at a time,
+// through TMA.
 //
 // "Wave Forcing: Towards Speed-of-Light Streaming Video Generation", Method
 // section: K/V are published right after the QKV projection and RoPE, and
