@@ -189,3 +189,28 @@ def test_mask_mode_validation():
         assert a.layout() == b.layout()
         a.advance()
         b.advance()
+
+
+def test_bench_traffic_record_follows_kernel_code(tmp_path):
+    # bench.py reports a kernel's recorded ncu traffic only while the hash of
+    # its code matches; comment and blank-line edits keep the hash.
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "bench_mod", os.path.join(os.path.dirname(os.path.dirname(__file__)), "bench.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    src = tmp_path / "k.cu"
+    src.write_text("// header\nint f(int x) {\n  return x + 1;   // add\n}\n")
+    h0 = b.source_sha(str(src))
+    src.write_text("// another header\n\nint f(int x) {\n  return x + 1;\n}\n")
+    assert b.source_sha(str(src)) == h0
+    src.write_text("int f(int x) {\n  return x + 2;\n}\n")
+    assert b.source_sha(str(src)) != h0
+    # every committed record matches the kernel source it names
+    import json
+    root = os.path.dirname(os.path.dirname(__file__))
+    rec = json.load(open(os.path.join(root, "profiles", "ncu_traffic.json")))
+    for key, e in rec.items():
+        path = os.path.join(root, "chunk_causal_wavefront_b200", "csrc", key.split(":")[0])
+        assert e["source_sha"] == b.source_sha(path), key
+        assert e["dram_bytes_per_launch"] > 0
