@@ -273,6 +273,24 @@ LiveSlots live_slots(const wf_pool *p) {
   return l;
 }
 
+// Keep only `slot` in the live list (slot < 0 keeps every slot); false if the
+// slot is not live in the current round.
+bool select_slot(LiveSlots &l, int32_t slot) {
+  if (slot < 0) return true;
+  for (int i = 0; i < l.n; ++i) {
+    if (l.slot[i] != slot) continue;
+    LiveSlots one{};
+    one.n = 1;
+    one.slot[0] = l.slot[i];
+    one.chunk[0] = l.chunk[i];
+    one.tag[0] = l.tag[i];
+    one.npos[0] = l.npos[i];
+    l = one;
+    return true;
+  }
+  return false;
+}
+
 bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
 bool on_pool_device(const wf_pool *p) {
@@ -402,8 +420,13 @@ wf_status wf_kv_pool_create(const wf_pool_config *cfg, void *dev_mem, size_t byt
   return WF_OK;
 }
 
-wf_status wf_publish_kv(wf_pool *p, int32_t layer, const void *q, const void *k, const void *v,
-                        void *q_rot, wf_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Publication of every live slot (only_slot < 0) or of one live slot.
+wf_status publish_impl(wf_pool *p, int32_t layer, const void *q, const void *k, const void *v,
+                       void *q_rot, int32_t only_slot, wf_stream_t stream) {
   if (!p) return WF_ERR_INVALID_ARG;
   if (p->host_only) return WF_ERR_CALL_ORDER;
   const wf_pool_config &c = p->cfg;
@@ -430,6 +453,8 @@ wf_status wf_publish_kv(wf_pool *p, int32_t layer, const void *q, const void *k,
   pp.rope = c.rope; pp.F = c.frames_per_chunk; pp.gh = c.grid_h; pp.gw = c.grid_w;
   pp.split0 = c.rope_split[0]; pp.split1 = c.rope_split[1]; pp.split2 = c.rope_split[2];
   pp.live = live_slots(p);
+  if (only_slot > c.num_stages) return WF_ERR_INVALID_ARG;
+  if (!select_slot(pp.live, only_slot)) return WF_ERR_CALL_ORDER;
   if (c.dtype == WF_DTYPE_FP8_E4M3) {
     pp.kv_scale = reinterpret_cast<float *>(p->dev + p->g.kv_scale_off) +
                   static_cast<size_t>(layer) * p->g.kv_scale_per_layer;
@@ -475,8 +500,10 @@ wf_status wf_publish_kv(wf_pool *p, int32_t layer, const void *q, const void *k,
   return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 
-wf_status wf_round_attention(wf_pool *p, int32_t layer, const void *q_rot, void *out,
-                             wf_stream_t stream) {
+// Round attention of every live slot (only_slot < 0) or of one live slot, whose
+// readiness check then covers only the context prefix it reads.
+wf_status attention_impl(wf_pool *p, int32_t layer, const void *q_rot, void *out,
+                         int32_t only_slot, wf_stream_t stream) {
   if (!p) return WF_ERR_INVALID_ARG;
   if (p->host_only) return WF_ERR_CALL_ORDER;
   const wf_pool_config &c = p->cfg;
@@ -498,6 +525,9 @@ wf_status wf_round_attention(wf_pool *p, int32_t layer, const void *q_rot, void 
   ap.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(c.head_dim)));
   ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
   ap.live = live_slots(p);
+  if (only_slot > c.num_stages) return WF_ERR_INVALID_ARG;
+  if (!select_slot(ap.live, only_slot)) return WF_ERR_CALL_ORDER;
+  if (only_slot >= 0) ap.n_pos = ap.live.npos[0];
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (c.dtype == WF_DTYPE_BF16 || c.dtype == WF_DTYPE_FP8_E4M3) {
@@ -534,6 +564,66 @@ wf_status wf_round_attention(wf_pool *p, int32_t layer, const void *q_rot, void 
   } else {
     e = launch_attention_f32(ap, cs);
   }
+  return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+wf_status wf_publish_kv(wf_pool *p, int32_t layer, const void *q, const void *k, const void *v,
+                        void *q_rot, wf_stream_t stream) {
+  return publish_impl(p, layer, q, k, v, q_rot, -1, stream);
+}
+
+wf_status wf_publish_kv_slot(wf_pool *p, int32_t layer, int32_t slot, const void *q,
+                             const void *k, const void *v, void *q_rot, wf_stream_t stream) {
+  if (slot < 0) return WF_ERR_INVALID_ARG;
+  return publish_impl(p, layer, q, k, v, q_rot, slot, stream);
+}
+
+wf_status wf_round_attention(wf_pool *p, int32_t layer, const void *q_rot, void *out,
+                             wf_stream_t stream) {
+  return attention_impl(p, layer, q_rot, out, -1, stream);
+}
+
+wf_status wf_round_attention_slot(wf_pool *p, int32_t layer, int32_t slot, const void *q_rot,
+                                  void *out, wf_stream_t stream) {
+  if (slot < 0) return WF_ERR_INVALID_ARG;
+  return attention_impl(p, layer, q_rot, out, slot, stream);
+}
+
+wf_status wf_deliver_kv(const wf_pool *p, int32_t layer, int32_t slot, void *dst_pool_mem,
+                        wf_stream_t stream) {
+  if (!p || !dst_pool_mem) return WF_ERR_INVALID_ARG;
+  if (p->host_only) return WF_ERR_CALL_ORDER;
+  const wf_pool_config &c = p->cfg;
+  if (layer < 0 || layer >= c.num_layers) return WF_ERR_INVALID_ARG;
+  if (slot < 0 || slot > c.num_stages) return WF_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(dst_pool_mem) & 255u) != 0) return WF_ERR_INVALID_ARG;
+  if (dst_pool_mem == p->dev) return WF_ERR_INVALID_ARG;
+  if (!on_pool_device(p)) return WF_ERR_INVALID_ARG;
+  LiveSlots l = live_slots(p);
+  if (!select_slot(l, slot)) return WF_ERR_CALL_ORDER;
+  char *dst = static_cast<char *>(dst_pool_mem);
+  const size_t page_off = p->g.pages_off + static_cast<size_t>(layer) * p->g.num_pages * p->g.page_bytes;
+  const size_t tag_off = p->g.tags_off + static_cast<size_t>(layer) * p->g.num_pages * sizeof(int32_t);
+  DeliverParams dp{};
+  dp.src_pages = p->dev + page_off;
+  dp.dst_pages = dst + page_off;
+  dp.src_tags = reinterpret_cast<const int32_t *>(p->dev + tag_off);
+  dp.dst_tags = reinterpret_cast<int32_t *>(dst + tag_off);
+  if (c.dtype == WF_DTYPE_FP8_E4M3) {
+    const size_t sc_off = p->g.kv_scale_off + static_cast<size_t>(layer) * p->g.kv_scale_per_layer * sizeof(float);
+    dp.src_kv_scale = reinterpret_cast<const float *>(p->dev + sc_off);
+    dp.dst_kv_scale = reinterpret_cast<float *>(dst + sc_off);
+  }
+  dp.table = reinterpret_cast<const int32_t *>(p->dev + p->g.table_off);
+  dp.status = reinterpret_cast<int32_t *>(p->dev + p->g.status_off);
+  dp.slot = slot; dp.npc = p->g.npc; dp.Hh = c.num_heads;
+  dp.num_pages = static_cast<int32_t>(p->g.num_pages); dp.tag = l.tag[0];
+  dp.tile_bytes = static_cast<int64_t>(c.page_tokens) * c.head_dim * p->g.elt;
+  const cudaError_t e = launch_deliver(dp, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? WF_OK : WF_ERR_CUDA;
 }
 

@@ -82,6 +82,21 @@ struct ProjectParams {
   LiveSlots live;
 };
 
+// One slot's pages of one layer, copied from this pool into a receiver pool of
+// the same geometry (same physical page ids), then the receiver's ready tags.
+struct DeliverParams {
+  const char *src_pages;      // this pool's page region of the layer
+  char *dst_pages;            // the receiver's page region of the layer
+  const int32_t *src_tags;    // this pool's ready tags of the layer
+  int32_t *dst_tags;          // the receiver's ready tags of the layer
+  const float *src_kv_scale;  // FP8 pools: this layer's [num_pages][2][heads] scales, else null
+  float *dst_kv_scale;        // FP8 pools: the receiver's, else null
+  const int32_t *table;       // this pool's device page table
+  int32_t *status;            // this pool's sticky status word
+  int32_t slot, npc, Hh, num_pages, tag;   // tag: the slot's ready tag this round
+  int64_t tile_bytes;         // one (page, K|V, head) tile: P * d * element size
+};
+
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_publish_f32(const PublishParams &p, cudaStream_t st);
 // The FP8 publish takes unswizzled tensor maps of q, k and v over
@@ -96,6 +111,7 @@ cudaError_t launch_publish_bf16_tma(const PublishParams &p, const void *tmap_q, 
                                     const void *tmap_v, const void *tmap_qrot,
                                     const void *tmap_pages, cudaStream_t st);
 cudaError_t launch_attention_f32(const AttnParams &p, cudaStream_t st);
+cudaError_t launch_deliver(const DeliverParams &p, cudaStream_t st);
 // The bf16 tensor-core path takes the encoded tensor maps (opaque 128-byte
 // CUtensorMap objects) of q_rot (box 64 x 1 x 128 rows), the pool's K/V pages
 // (box 64 x 128) and out (box 64 x 1 x 32 rows).

@@ -103,6 +103,30 @@ class KVPool:
         if st != _wf.WF_OK:
             raise WfError(st, "wf_round_attention")
 
+    # -- Wave Parallelism: one slot per rank ------------------------------------------
+    def publish_slot(self, layer: int, slot: int, q: torch.Tensor, k: torch.Tensor,
+                     v: torch.Tensor, q_rot: torch.Tensor, stream=None) -> None:
+        st = _wf.wf_publish_kv_slot(self.handle, layer, slot, _ptr(q), _ptr(k), _ptr(v),
+                                    _ptr(q_rot), _stream(self.device, stream))
+        if st != _wf.WF_OK:
+            raise WfError(st, "wf_publish_kv_slot")
+
+    def attention_slot(self, layer: int, slot: int, q_rot: torch.Tensor, out: torch.Tensor,
+                       stream=None) -> None:
+        st = _wf.wf_round_attention_slot(self.handle, layer, slot, _ptr(q_rot), _ptr(out),
+                                         _stream(self.device, stream))
+        if st != _wf.WF_OK:
+            raise WfError(st, "wf_round_attention_slot")
+
+    def deliver(self, layer: int, slot: int, dst: "KVPool", stream=None) -> None:
+        """Copy this pool's pages of `slot` (published in this round) into the
+        receiver pool `dst` (same config, page order and round) and stamp its
+        ready tags. `dst.mem` must be addressable from this pool's device."""
+        st = _wf.wf_deliver_kv(self.handle, layer, slot, dst.mem.data_ptr(),
+                               _stream(self.device, stream))
+        if st != _wf.WF_OK:
+            raise WfError(st, "wf_deliver_kv")
+
     def advance(self, stream=None) -> None:
         s = 0 if self.device is None else _stream(self.device, stream)
         st = _wf.wf_advance_round(self.handle, s)

@@ -35,7 +35,7 @@ EXPORTS = (
     "wf_kv_pool_bytes", "wf_kv_pool_create", "wf_publish_kv", "wf_round_attention",
     "wf_advance_round", "wf_pool_check_status", "wf_pool_destroy", "wf_status_string",
     "wf_pool_round", "wf_pool_get_geometry", "wf_pool_get_layout", "wf_pool_debug_poke_page",
-    "wf_project_publish",
+    "wf_project_publish", "wf_publish_kv_slot", "wf_round_attention_slot", "wf_deliver_kv",
 )
 
 
@@ -93,6 +93,9 @@ def _load():
         "wf_pool_get_layout": (I32, [P, i32p, i32p, i32p, i32p, i32p, i32p, I32]),
         "wf_pool_debug_poke_page": (I32, [P, I32, I32, I32, P]),
         "wf_project_publish": (I32, [P, I32, P, P, P, P]),
+        "wf_publish_kv_slot": (I32, [P, I32, I32, P, P, P, P, P]),
+        "wf_round_attention_slot": (I32, [P, I32, I32, P, P, P]),
+        "wf_deliver_kv": (I32, [P, I32, I32, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -141,6 +144,22 @@ def wf_publish_kv(pool: int, layer: int, q: int, k: int, v: int, q_rot: int, str
 
 def wf_round_attention(pool: int, layer: int, q_rot: int, out: int, stream: int) -> int:
     return _lib.wf_round_attention(pool, layer, q_rot, out, ctypes.c_void_p(stream or None))
+
+
+def wf_publish_kv_slot(pool: int, layer: int, slot: int, q: int, k: int, v: int, q_rot: int,
+                       stream: int) -> int:
+    return _lib.wf_publish_kv_slot(pool, layer, slot, q, k, v, q_rot,
+                                   ctypes.c_void_p(stream or None))
+
+
+def wf_round_attention_slot(pool: int, layer: int, slot: int, q_rot: int, out: int,
+                            stream: int) -> int:
+    return _lib.wf_round_attention_slot(pool, layer, slot, q_rot, out,
+                                        ctypes.c_void_p(stream or None))
+
+
+def wf_deliver_kv(pool: int, layer: int, slot: int, dst_pool_mem: int, stream: int) -> int:
+    return _lib.wf_deliver_kv(pool, layer, slot, dst_pool_mem, ctypes.c_void_p(stream or None))
 
 
 def wf_advance_round(pool: int, stream: int) -> int:

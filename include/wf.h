@@ -176,6 +176,55 @@ wf_status wf_publish_kv(wf_pool *pool, int32_t layer, const void *q, const void 
 wf_status wf_round_attention(wf_pool *pool, int32_t layer, const void *q_rot, void *out,
                              wf_stream_t stream);
 
+/* Wave Parallelism (Method section, Figure 3c; thelatestinai listing, Table
+ * 10): one GPU per stage, each running one query slot per round, with one-way
+ * K/V delivery into the pages of the stages that read them and a ready signal.
+ * Every rank keeps a full pool created with the same config and page_order and
+ * advanced through the same rounds, so the page tables (and the physical ids
+ * of every slot's pages) are the same on all ranks. A round on rank r, owner
+ * of slot r (the store rank owns slot S):
+ *   wf_publish_kv_slot(r) -> wf_deliver_kv(r) to each reader ->
+ *   wf_round_attention_slot(r) once the deliveries into this pool have landed
+ *   (the caller orders them, e.g. with a barrier or an IPC event);
+ * readers of slot j are the live slots s < j under WF_MASK_WF, every live slot
+ * under WF_MASK_RF, and every rank for the store (its chunk becomes anchor or
+ * history for all later rounds). wave_plan() in the Python binding lists them.
+ *
+ * wf_publish_kv_slot: wf_publish_kv restricted to one live slot: reads only
+ * that slot's rows of q, k, v ([S+1][C][heads][d] buffers), writes its q_rot
+ * rows, its pages and their ready tags. WF_ERR_CALL_ORDER if the slot is not
+ * live in this round. */
+wf_status wf_publish_kv_slot(wf_pool *pool, int32_t layer, int32_t slot, const void *q,
+                             const void *k, const void *v, void *q_rot, wf_stream_t stream);
+
+/* wf_round_attention restricted to one live query slot: writes only that
+ * slot's rows of out, and checks the ready tags of only the context prefix the
+ * slot reads (under WF_MASK_RF, the whole context). WF_ERR_CALL_ORDER if the
+ * slot is not live in this round. */
+wf_status wf_round_attention_slot(wf_pool *pool, int32_t layer, int32_t slot, const void *q_rot,
+                                  void *out, wf_stream_t stream);
+
+/* Deliver one live slot's published K/V pages of one layer into a receiver's
+ * pool: every (page, K|V, head) tile of the slot's chunk (and, for FP8_E4M3
+ * pools, its block scale) is copied to the same physical page of the
+ * receiver, then the receiver's ready tags of those pages are set to the
+ * slot's tag of this round.
+ *   dst_pool_mem : the receiver pool's device buffer (as passed to its
+ *                  wf_kv_pool_create), 256-byte aligned and addressable from
+ *                  the current device: a buffer on this device or a peer
+ *                  device's buffer with peer access enabled (the copy stores
+ *                  go over NVLink). The receiver must have this pool's config,
+ *                  page order and round (not checked: the receiver may be on
+ *                  another process's device).
+ * The kernels first check this pool's page ids and ready tags for the slot: a
+ * bad id records WF_ERR_BAD_PAGE, a tag from another round WF_ERR_NOT_READY
+ * (the slot was not published in this round), in this pool's status word, and
+ * nothing is written to the receiver. The tags are written by a second kernel
+ * in stream order after the data. WF_ERR_CALL_ORDER if the slot is not live;
+ * WF_ERR_INVALID_ARG for a NULL, misaligned or self receiver buffer. */
+wf_status wf_deliver_kv(const wf_pool *pool, int32_t layer, int32_t slot, void *dst_pool_mem,
+                        wf_stream_t stream);
+
 /* Fused QKV projection + publication for one layer (Method section: the local
  * QKV projection runs without waiting for remote K/V, and K/V are published
  * right after the projection and RoPE, written straight into the ordered
