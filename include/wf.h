@@ -18,7 +18,9 @@
  *
  * Conventions for every call:
  *   - Pointers named q, k, v, q_rot, out and dev_mem are DEVICE pointers on the
- *     current CUDA device; config structs and page_order are HOST pointers.
+ *     current CUDA device; dst_pool_mem (wf_deliver_kv) is a device pointer
+ *     addressable from it (its own memory or a peer device's); config structs
+ *     and page_order are HOST pointers.
  *   - Activations are laid out [S+1][C][num_heads][head_dim], row-major, in the
  *     pool's dtype (bf16 or fp32; FP8 pools: see WF_DTYPE_FP8_E4M3): slot-major,
  *     then token, head, dimension.
