@@ -114,3 +114,86 @@ def test_plan_on_gloo_ranks(world):
                 j = lay[i].slot
                 if j is not None and j != s:
                     assert (k, j) in received[s], (k, s, j)
+
+
+# Delivery writes a slot's pages at the same physical ids in the receiver's
+# pool, which holds only because every rank's bookkeeping is the same
+# function of (config, page order, round). Host-only pools (no device memory)
+# run that bookkeeping here.
+def _layouts(cfg, order, rounds):
+    import chunk_causal_wavefront_b200 as wfb
+    from wf_test_utils import pool_config
+    pool = wfb.KVPool(pool_config(cfg, max_rounds=rounds + 2), page_order=order)
+    out = []
+    for _ in range(rounds):
+        out.append(pool.layout())
+        pool.advance()
+    pool.close()
+    return out
+
+
+def test_rank_pools_keep_identical_page_tables():
+    import wf_inputs
+    from wf_test_utils import min_pages
+    cfg = wf_inputs.CONFIGS["wan13b_bf16"]
+    order = wf_inputs.draw_page_order(min_pages(cfg), 5)
+    ranks = [_layouts(cfg, order, 60) for _ in range(cfg.num_stages + 1)]
+    assert all(r == ranks[0] for r in ranks)
+    # and the pages the plan hands over in a steady round are the slot's own pages
+    lay = ranks[0][cfg.steady_round()]
+    pages = {slot: pg for kind, chunk, slot, tag, pg in lay if slot is not None and slot >= 0}
+    assert sorted(pages) == live_slots(cfg.num_stages, cfg.steady_round())
+    flat = [p for pg in pages.values() for p in pg]
+    assert len(flat) == len(set(flat))                    # no page shared between slots
+
+
+def test_wave_calls_on_host_only_pools():
+    import wf_inputs
+    import chunk_causal_wavefront_b200 as wfb
+    from chunk_causal_wavefront_b200 import wf as W
+    from wf_test_utils import pool_config
+    cfg = wf_inputs.CONFIGS["tiny_f32"]
+    pool = wfb.KVPool(pool_config(cfg))
+    assert W.wf_publish_kv_slot(pool.handle, 0, 0, 16, 16, 16, 32, 0) == W.WF_ERR_CALL_ORDER
+    assert W.wf_publish_kv_slot(pool.handle, 0, -1, 16, 16, 16, 32, 0) == W.WF_ERR_INVALID_ARG
+    assert W.wf_round_attention_slot(pool.handle, 0, 0, 16, 32, 0) == W.WF_ERR_CALL_ORDER
+    assert W.wf_round_attention_slot(pool.handle, 0, -1, 16, 32, 0) == W.WF_ERR_INVALID_ARG
+    assert W.wf_deliver_kv(pool.handle, 0, 0, 256, 0) == W.WF_ERR_CALL_ORDER
+    assert W.wf_deliver_kv(pool.handle, 0, 0, None, 0) == W.WF_ERR_INVALID_ARG
+    assert W.lib().wf_deliver_kv(None, 0, 0, None, None) == W.WF_ERR_INVALID_ARG
+    pool.close()
+
+
+def _rank_tables(rank, world, port, q):
+    import hashlib
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import wf_inputs
+    from wf_test_utils import min_pages
+    cfg = wf_inputs.CONFIGS["wan13b_bf16"].replace(num_stages=world - 1)
+    order = wf_inputs.draw_page_order(min_pages(cfg), 11)
+    digest = [hashlib.sha256(repr(l).encode()).hexdigest() for l in _layouts(cfg, order, 40)]
+    got = [None] * world
+    dist.all_gather_object(got, digest)
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, got))
+
+
+def test_page_tables_agree_across_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    world = 3
+    port = 29700 + os.getpid() % 1000
+    procs = [ctx.Process(target=_rank_tables, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in range(world):
+        assert all(d == res[r][0] for d in res[r])         # all ranks: same tables, every round
