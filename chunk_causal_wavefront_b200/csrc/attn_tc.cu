@@ -52,8 +52,9 @@
 //         sub-partition and tile; the turn passes after three quarters of the
 //         row).
 // Every wait is bounded: on timeout the CTA records WF_ERR_TIMEOUT, the other
-// roles see the abort flag, in-flight copies and MMAs are drained and TMEM is
-// freed before the CTA exits.
+// roles see the abort flag, in-flight copies and MMAs are drained (with a
+// separate, longer bound), pending TMEM stores are waited for, and TMEM is
+// freed before the CTA exits. No output of a CTA that gave up is written.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -122,6 +123,47 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+#ifndef WF_F8_POLY_PAIRS
+#define WF_F8_POLY_PAIRS 6
+#endif
+#ifndef WF_F8_TURNS
+#define WF_F8_TURNS 1
+#endif
+// E4M3: of every 16 pairs of exponentials, this many run as a polynomial on
+// the FMA pipe instead of the MUFU unit (which does 16 exponentials per clock
+// per SM, in the f32 form as in the packed f16x2/bf16x2 forms: measured).
+constexpr int kF8PolyPairs = WF_F8_POLY_PAIRS;
+constexpr bool kF8Turns = WF_F8_TURNS != 0;
+
+// 2^x for a pair of values on the FMA pipe: x = n + f with n = round(x) (adding
+// and subtracting 1.5 * 2^23 rounds to an integer) and f in [-1/2, 1/2]; 2^f
+// from a degree-2 polynomial whose coefficients minimise the largest relative
+// error on [-1/2, 1/2] (1.73e-3, far below E4M3's half unit of 2^-4); n is
+// added to the exponent field. x is clamped below at -127 first, so -inf
+// (masked keys) and very small probabilities come out as 2^-127 or less,
+// which rounds to zero in E4M3 at any block scale the kernel uses.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float a, b;
+  unf2(x2, a, b);
+  const uint64_t xc = f2(fmaxf(a, -127.0f), fmaxf(b, -127.0f));
+  const uint64_t t = fadd2(xc, f2(12582912.0f, 12582912.0f));    // 1.5 * 2^23 + n
+  float t0, t1;
+  unf2(t, t0, t1);
+  const uint64_t nf = fadd2(t, f2(-12582912.0f, -12582912.0f));  // n
+  float n0, n1;
+  unf2(nf, n0, n1);
+  const uint64_t fr = fadd2(xc, f2(-n0, -n1));                    // f
+  uint64_t p = ffma2(fr, f2(0.23842734f, 0.23842734f), f2(0.70344603f, 0.70344603f));
+  p = ffma2(p, fr, f2(1.0004431f, 1.0004431f));
+  float p0, p1;
+  unf2(p, p0, p1);
+  // the low bits of t's pattern hold n (two's complement); shifted into the
+  // exponent field they scale p by 2^n
+  p0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+  return f2(p0, p1);
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -282,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const Ctx ctx{bars, abort_flag, p.status};
+  const Ctx ctx{bars, abort_flag, p.status, p.wait_limit};
   const int last_valid = p.C - (p.npc - 1) * p.P;   // keys in a chunk's last page
 
   if (warp >= 8) {
@@ -316,10 +358,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t *sK = smem + F::kOffK + stg * kTile;
         uint8_t *sV = smem + F::kOffV + stg * kTile;
         if (!wait_bar(ctx, kKEmpty0 + stg, ph ^ 1)) break;
-        mbar_arrive_expect_tx(bars + kKFull0 + stg, kTile);
-        tma_load_2d(sK, &tkv, bars + kKFull0 + stg, 0, rowk);
-        if (!kF8) tma_load_2d(sK + F::kHalf, &tkv, bars + kKFull0 + stg, 64, rowk);
-        if (stg) ++nk1; else ++nk0;
+        if (j != p.skip_key_tile) {   // test hook: a skipped load leaves its wait to run out
+          mbar_arrive_expect_tx(bars + kKFull0 + stg, kTile);
+          tma_load_2d(sK, &tkv, bars + kKFull0 + stg, 0, rowk);
+          if (!kF8) tma_load_2d(sK + F::kHalf, &tkv, bars + kKFull0 + stg, 64, rowk);
+          if (stg) ++nk1; else ++nk0;
+        }
         if (!wait_bar(ctx, kVEmpty0 + stg, ph ^ 1)) break;
         mbar_arrive_expect_tx(bars + kVFull0 + stg, kTile);
         tma_load_2d(sV, &tkv, bars + kVFull0 + stg, 0, rowv);
@@ -327,6 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (stg) ++nv1; else ++nv0;
       }
       // Drain: every load this thread issued has landed before the CTA exits.
+      // Loads into one stage complete its phases in order, so waiting for the
+      // phase of the last one issued covers them all.
       if (nk0) drain_wait(ctx, kKFull0, (nk0 - 1) & 1);
       if (nk1) drain_wait(ctx, kKFull0 + 1, (nk1 - 1) & 1);
       if (nv0) drain_wait(ctx, kVFull0, (nv0 - 1) & 1);
@@ -462,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // to itself; the turn is handed on after three quarters of the row. With
       // the FP8 MMAs' shorter P*V + S the two phases would otherwise overlap
       // (bf16 tiles stay apart by themselves, and a turn only delays them).
-      if (kF8 && has_q1 && (q == 1 || j > 0)) {
+      if (kF8 && kF8Turns && has_q1 && (q == 1 || j > 0)) {
         ok = __all_sync(0xffffffffu, wait_bar(ctx, (q == 0 ? kTurn0 : kTurn1) + (warp & 3),
                                               q == 0 ? ((j - 1) & 1) : (j & 1)));
         if (!ok) break;
@@ -477,16 +523,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 16; ++c) {
             const int k0 = cc * 32 + 2 * c;
             const uint64_t x2 = ffma2(f2(__uint_as_float(s[k0]), __uint_as_float(s[k0 + 1])), sc2, nm2);
-            float a, b;
-            unf2(x2, a, b);
-            const float e0 = ex2(a), e1 = ex2(b);
+            float e0, e1;
+            if (c % 8 >= 8 - kF8PolyPairs / 2 - (c < 8 ? kF8PolyPairs % 2 : 0)) {
+              unf2(exp2_poly2(x2), e0, e1);
+            } else {
+              float a, b;
+              unf2(x2, a, b);
+              e0 = ex2(a);
+              e1 = ex2(b);
+            }
             acc[c & 3] = fadd2(acc[c & 3], f2(e0, e1));
             const uint32_t pr = pack_e4m3x2(e0, e1);
             if (c & 1) pw[c >> 1] = join16(half, pr);
             else half = pr;
           }
           tmem_st8(tS + cc * 8, pw);
-          if (cc == 2 && has_q1 && lane == 0)
+          if (kF8Turns && cc == 2 && has_q1 && lane == 0)
             mbar_arrive(bars + (q == 0 ? kTurn1 : kTurn0) + (warp & 3));
         } else {
           uint32_t pw[16];
@@ -587,6 +639,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
+    // A softmax that gave up mid-tile may still have TMEM stores in flight.
+    tmem_st_wait();
    }
   }
 

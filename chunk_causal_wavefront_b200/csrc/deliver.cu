@@ -17,12 +17,17 @@
 //     tile; 16-byte loads from this pool, 16-byte stores into the receiver's
 //     pool (a peer device's memory over NVLink, or this device's); FP8 pools
 //     also copy the tile's block scale. A system-scope fence ends each CTA.
-//   * deliver_tags_kernel: writes the receiver's ready tags of the slot's pages
-//     once every tile has landed (stream order after the copy kernel).
-// Both first check, in every CTA, that all of the slot's page ids are in range
-// and that this pool's tags say the slot was published in this round; a bad id
-// records WF_ERR_BAD_PAGE, a stale tag WF_ERR_NOT_READY, and nothing is
-// written to the receiver.
+//     Each CTA first checks the receiver's pool signature (config and page
+//     order, written at pool creation) and its own page: an id in range whose
+//     ready tag in this pool is this round's. A foreign receiver records
+//     WF_ERR_INVALID_ARG, a bad id WF_ERR_BAD_PAGE, a stale tag
+//     WF_ERR_NOT_READY, and the CTA writes nothing.
+//   * deliver_tags_kernel: checks every page of the slot the same way, and
+//     only if all pass writes the receiver's ready tags of the slot's pages
+//     (stream order after the copy kernel, so after every tile has landed).
+// So a receiver's tags are stamped only for a slot whose every page was
+// published in this round and copied; a slot that was not published at all
+// leaves the receiver untouched.
 #include "wf_internal.h"
 
 namespace wf {
@@ -30,34 +35,35 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// 0 if every page of the slot is in range and carries the expected tag, else
-// the status to record. Every thread of the CTA returns the same value.
-__device__ __forceinline__ int check_slot_pages(const DeliverParams &p, int pos) {
-  int bad = 0, stale = 0;
-  for (int j = threadIdx.x; j < p.npc; j += blockDim.x) {
-    const int pg = __ldcg(p.table + kTabPages + pos * p.npc + j);
-    if (pg < 0 || pg >= p.num_pages) bad = 1;
-    else if (__ldcg(p.src_tags + pg) != p.tag) stale = 1;
-  }
-  const int any_bad = __syncthreads_or(bad);
-  const int any_stale = __syncthreads_or(stale);
-  return any_bad ? WF_ERR_BAD_PAGE : (any_stale ? WF_ERR_NOT_READY : 0);
+// 0 if page j of the slot is in range and carries the expected tag, else the
+// status to record.
+__device__ __forceinline__ int check_page(const DeliverParams &p, int pos, int j) {
+  const int pg = __ldcg(p.table + kTabPages + pos * p.npc + j);
+  if (pg < 0 || pg >= p.num_pages) return WF_ERR_BAD_PAGE;
+  if (__ldcg(p.src_tags + pg) != p.tag) return WF_ERR_NOT_READY;
+  return 0;
 }
 
 __global__ void __launch_bounds__(kThreads) deliver_copy_kernel(const DeliverParams p) {
   const int j = blockIdx.x;                  // page of the slot's chunk
   const int kvh = blockIdx.y;                // K|V x head: kv * heads + h
-  const int pos = __ldcg(p.table + kTabSlotPos + p.slot);
-  if (pos < 0) {
-    if (threadIdx.x == 0) record_status(p.status, WF_ERR_BAD_PAGE);
-    return;
+  __shared__ int verdict;
+  if (threadIdx.x == 0) {
+    const int pos = __ldcg(p.table + kTabSlotPos + p.slot);
+    int st = 0;
+    if (*reinterpret_cast<const volatile uint64_t *>(p.dst_signature) != p.signature)
+      st = WF_ERR_INVALID_ARG;
+    else if (pos < 0)
+      st = WF_ERR_BAD_PAGE;
+    else
+      st = check_page(p, pos, j);
+    // one CTA per page records its page's problem (the K|V x head CTAs agree)
+    if (st && kvh == 0) record_status(p.status, st);
+    verdict = st ? -1 : __ldcg(p.table + kTabPages + pos * p.npc + j);
   }
-  const int st = check_slot_pages(p, pos);
-  if (st) {
-    if (threadIdx.x == 0 && j == 0 && kvh == 0) record_status(p.status, st);
-    return;
-  }
-  const int phys = __ldcg(p.table + kTabPages + pos * p.npc + j);
+  __syncthreads();
+  const int phys = verdict;
+  if (phys < 0) return;
   const size_t tile = static_cast<size_t>(phys) * 2 * p.Hh + kvh;
   const uint4 *src = reinterpret_cast<const uint4 *>(p.src_pages + tile * p.tile_bytes);
   uint4 *dst = reinterpret_cast<uint4 *>(p.dst_pages + tile * p.tile_bytes);
@@ -68,9 +74,12 @@ __global__ void __launch_bounds__(kThreads) deliver_copy_kernel(const DeliverPar
 }
 
 __global__ void __launch_bounds__(kThreads) deliver_tags_kernel(const DeliverParams p) {
+  if (*reinterpret_cast<const volatile uint64_t *>(p.dst_signature) != p.signature) return;
   const int pos = __ldcg(p.table + kTabSlotPos + p.slot);
   if (pos < 0) return;                       // recorded by the copy kernel
-  if (check_slot_pages(p, pos)) return;      // idem
+  int bad = 0;
+  for (int j = threadIdx.x; j < p.npc; j += kThreads) bad |= check_page(p, pos, j);
+  if (__syncthreads_or(bad)) return;         // idem
   for (int j = threadIdx.x; j < p.npc; j += kThreads)
     p.dst_tags[__ldcg(p.table + kTabPages + pos * p.npc + j)] = p.tag;
   __threadfence_system();

@@ -181,9 +181,46 @@ bool encode_plain_bf16_map(CUtensorMap *map, void *base, int rank, const cuuint6
   return r == CUDA_SUCCESS;
 }
 
+// Unswizzled tiled map over bytes (E4M3 codes).
+bool encode_plain_u8_map(CUtensorMap *map, void *base, int rank, const cuuint64_t *dims,
+                         const cuuint64_t *strides_bytes, const cuuint32_t *box) {
+  auto fn = get_encode();
+  if (!fn) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, base, dims, strides_bytes, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool encode_bf16_map(CUtensorMap *map, void *base, int rank, const cuuint64_t *dims,
                      const cuuint64_t *strides_bytes, const cuuint32_t *box) {
   return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box);
+}
+
+// 64-bit FNV-1a over the bytes of the config (its fields, one by one, so
+// that struct padding does not enter), the initial page order and the pool
+// size: pools that deliver into each other must agree on all three.
+uint64_t pool_signature(const wf_pool_config &c, const std::vector<int32_t> &order, size_t total) {
+  uint64_t h = 1469598103934665603ULL;
+  auto mix = [&h](const void *data, size_t n) {
+    const unsigned char *b = static_cast<const unsigned char *>(data);
+    for (size_t i = 0; i < n; ++i) {
+      h ^= b[i];
+      h *= 1099511628211ULL;
+    }
+  };
+  const int32_t words[] = {c.num_stages, c.chunk_tokens, c.num_heads, c.head_dim,
+                           c.anchor_chunks, c.history_chunks, c.page_tokens, c.num_layers,
+                           c.dtype, c.rope, c.frames_per_chunk, c.grid_h, c.grid_w,
+                           c.rope_split[0], c.rope_split[1], c.rope_split[2], c.max_rounds,
+                           c.num_pages, c.mask_mode};
+  mix(words, sizeof(words));
+  mix(&c.rope_base, sizeof(c.rope_base));
+  mix(order.data(), order.size() * sizeof(int32_t));
+  const uint64_t t = total;
+  mix(&t, sizeof(t));
+  return h ? h : 1;
 }
 
 }  // namespace
@@ -191,6 +228,7 @@ bool encode_bf16_map(CUtensorMap *map, void *base, int rank, const cuuint64_t *d
 struct wf_pool {
   wf_pool_config cfg{};
   Geometry g;
+  uint64_t signature = 0;   // config + page order, also stored in the device memory
   bool host_only = false;
   char *dev = nullptr;
   int device = -1;
@@ -204,6 +242,10 @@ struct wf_pool {
   std::deque<std::pair<int, std::vector<int32_t>>> history;
   std::vector<Position> layout;                   // current ordered context
   CUtensorMap kv_map;                             // bf16 / E4M3 pages, 2D rows x d
+  // Test hook (wf_pool_debug_stall_next_attention), consumed by the next
+  // tensor-core attention launch.
+  int32_t stall_key_tile = -1;
+  long long stall_wait_limit = 0;
 };
 
 namespace {
@@ -357,6 +399,7 @@ wf_status wf_kv_pool_create(const wf_pool_config *cfg, void *dev_mem, size_t byt
   p->g = g;
   p->host_only = host_only;
   p->dev = static_cast<char *>(dev_mem);
+  p->signature = pool_signature(*cfg, order, g.total);
   p->free_list.assign(order.begin(), order.end());
   const int S = cfg->num_stages;
   p->slot_pages.resize(S);
@@ -371,6 +414,10 @@ wf_status wf_kv_pool_create(const wf_pool_config *cfg, void *dev_mem, size_t byt
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     if (cudaGetDevice(&p->device) != cudaSuccess) { delete p; return WF_ERR_CUDA; }
     cudaError_t e = cudaMemsetAsync(p->dev, 0, g.pages_off, cs);   // status, table, tags
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(p->dev + g.status_off + kSignatureOffset, &p->signature,
+                          sizeof(p->signature), cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);   // the signature's source is on this stack
     if (e == cudaSuccess && cfg->rope == WF_ROPE_3D) {
       // (cos, sin) of angle = pos * base^(-2m / width), in float64, rounded to fp32.
       const int widths[3] = {cfg->rope_split[0], cfg->rope_split[1], cfg->rope_split[2]};
@@ -479,7 +526,13 @@ wf_status publish_impl(wf_pool *p, int32_t layer, const void *q, const void *k, 
         !encode_plain_bf16_map(&mv, const_cast<void *>(v), 4, dims, strides, box))
       return WF_ERR_CUDA;
     if (c.dtype == WF_DTYPE_FP8_E4M3) {
-      e = launch_publish_fp8(pp, &mq, &mk, &mv, cs);
+      // q_rot codes: [S+1][C][heads][d] bytes, one box = a 128-row tile of one head
+      const cuuint64_t cstr[3] = {static_cast<cuuint64_t>(c.head_dim),
+                                  static_cast<cuuint64_t>(c.head_dim) * c.num_heads,
+                                  static_cast<cuuint64_t>(c.head_dim) * c.num_heads * c.chunk_tokens};
+      CUtensorMap mqr;
+      if (!encode_plain_u8_map(&mqr, q_rot, 4, dims, cstr, box)) return WF_ERR_CUDA;
+      e = launch_publish_fp8(pp, &mq, &mk, &mv, &mqr, cs);
     } else {
       // q_rot as the inputs; the layer's pages as [pages x 2 x heads x P rows][d],
       // box 64 rows.
@@ -528,6 +581,13 @@ wf_status attention_impl(wf_pool *p, int32_t layer, const void *q_rot, void *out
   if (only_slot > c.num_stages) return WF_ERR_INVALID_ARG;
   if (!select_slot(ap.live, only_slot)) return WF_ERR_CALL_ORDER;
   if (only_slot >= 0) ap.n_pos = ap.live.npos[0];
+  ap.wait_limit = 2000000000LL;   // ~1 s at 2 GHz
+  ap.skip_key_tile = -1;
+  if (p->stall_key_tile >= 0 && c.dtype != WF_DTYPE_F32) {
+    ap.skip_key_tile = p->stall_key_tile;
+    ap.wait_limit = p->stall_wait_limit;
+    p->stall_key_tile = -1;
+  }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (c.dtype == WF_DTYPE_BF16 || c.dtype == WF_DTYPE_FP8_E4M3) {
@@ -594,9 +654,10 @@ wf_status wf_round_attention_slot(wf_pool *p, int32_t layer, int32_t slot, const
 }
 
 wf_status wf_deliver_kv(const wf_pool *p, int32_t layer, int32_t slot, void *dst_pool_mem,
-                        wf_stream_t stream) {
+                        size_t dst_pool_bytes, wf_stream_t stream) {
   if (!p || !dst_pool_mem) return WF_ERR_INVALID_ARG;
   if (p->host_only) return WF_ERR_CALL_ORDER;
+  if (dst_pool_bytes != p->g.total) return WF_ERR_INVALID_ARG;
   const wf_pool_config &c = p->cfg;
   if (layer < 0 || layer >= c.num_layers) return WF_ERR_INVALID_ARG;
   if (slot < 0 || slot > c.num_stages) return WF_ERR_INVALID_ARG;
@@ -620,6 +681,8 @@ wf_status wf_deliver_kv(const wf_pool *p, int32_t layer, int32_t slot, void *dst
   }
   dp.table = reinterpret_cast<const int32_t *>(p->dev + p->g.table_off);
   dp.status = reinterpret_cast<int32_t *>(p->dev + p->g.status_off);
+  dp.dst_signature = reinterpret_cast<const uint64_t *>(dst + p->g.status_off + kSignatureOffset);
+  dp.signature = p->signature;
   dp.slot = slot; dp.npc = p->g.npc; dp.Hh = c.num_heads;
   dp.num_pages = static_cast<int32_t>(p->g.num_pages); dp.tag = l.tag[0];
   dp.tile_bytes = static_cast<int64_t>(c.page_tokens) * c.head_dim * p->g.elt;
@@ -775,6 +838,18 @@ wf_status wf_pool_get_layout(const wf_pool *p, int32_t *n_positions, int32_t *ki
     if (pages)
       for (int j = 0; j < p->g.npc; ++j) pages[i * p->g.npc + j] = q.pages[j];
   }
+  return WF_OK;
+}
+
+wf_status wf_pool_debug_stall_next_attention(wf_pool *p, int32_t key_tile,
+                                             int64_t wait_limit_cycles) {
+  if (!p) return WF_ERR_INVALID_ARG;
+  if (p->host_only) return WF_ERR_CALL_ORDER;
+  if (p->cfg.dtype == WF_DTYPE_F32) return WF_ERR_UNSUPPORTED;
+  if (key_tile < 0 || wait_limit_cycles < 1000 || wait_limit_cycles > 2000000000LL)
+    return WF_ERR_INVALID_ARG;
+  p->stall_key_tile = key_tile;
+  p->stall_wait_limit = wait_limit_cycles;
   return WF_OK;
 }
 

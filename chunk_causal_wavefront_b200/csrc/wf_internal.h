@@ -66,6 +66,8 @@ struct AttnParams {
   const float *q_scale;       // FP8 pool: this layer's [S+1][npc][heads] query-tile scales
   float scale_log2;           // log2(e) / sqrt(d)
   float scale;                // 1 / sqrt(d)
+  long long wait_limit;       // cycles before a bounded wait gives up (tensor-core path)
+  int32_t skip_key_tile;      // test hook: key tile whose K load is never issued, else -1
   LiveSlots live;
 };
 
@@ -93,16 +95,24 @@ struct DeliverParams {
   float *dst_kv_scale;        // FP8 pools: the receiver's, else null
   const int32_t *table;       // this pool's device page table
   int32_t *status;            // this pool's sticky status word
+  const uint64_t *dst_signature;   // the receiver's pool signature word
+  uint64_t signature;         // this pool's signature (config and page order)
   int32_t slot, npc, Hh, num_pages, tag;   // tag: the slot's ready tag this round
   int64_t tile_bytes;         // one (page, K|V, head) tile: P * d * element size
 };
 
+// Byte offset, inside the pool memory's 256-byte status region, of the 64-bit
+// signature of the pool's config and page order, written at creation.
+constexpr size_t kSignatureOffset = 8;
+
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_publish_f32(const PublishParams &p, cudaStream_t st);
 // The FP8 publish takes unswizzled tensor maps of q, k and v over
-// [S+1][C][heads][d] bf16 with a box of 128 dims x 1 head x 128 rows.
+// [S+1][C][heads][d] bf16 with a box of 128 dims x 1 head x 128 rows, and an
+// unswizzled map of the q_rot codes over [S+1][C][heads][d] bytes with the
+// same box.
 cudaError_t launch_publish_fp8(const PublishParams &p, const void *tmap_q, const void *tmap_k,
-                               const void *tmap_v, cudaStream_t st);
+                               const void *tmap_v, const void *tmap_qrot, cudaStream_t st);
 // The bf16 publish for d = 128 and 128-token pages takes unswizzled maps of q,
 // k, v and q_rot over [S+1][C][heads][d] bf16 with a box of 128 dims x 1 head x
 // 64 rows, and an unswizzled 2D map over the layer's pool rows

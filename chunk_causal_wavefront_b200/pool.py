@@ -122,10 +122,27 @@ class KVPool:
         """Copy this pool's pages of `slot` (published in this round) into the
         receiver pool `dst` (same config, page order and round) and stamp its
         ready tags. `dst.mem` must be addressable from this pool's device."""
-        st = _wf.wf_deliver_kv(self.handle, layer, slot, dst.mem.data_ptr(),
+        self.deliver_to(layer, slot, dst.mem.data_ptr(), dst.nbytes, stream)
+
+    def deliver_to(self, layer: int, slot: int, dst_pool_mem: int, dst_pool_bytes: int,
+                   stream=None) -> None:
+        """wf_deliver_kv into a receiver given by its raw device pointer and size,
+        e.g. another process's pool buffer mapped with wf_ipc_open_mem."""
+        st = _wf.wf_deliver_kv(self.handle, layer, slot, dst_pool_mem, dst_pool_bytes,
                                _stream(self.device, stream))
         if st != _wf.WF_OK:
             raise WfError(st, "wf_deliver_kv")
+
+    def ipc_handle(self):
+        """(handle bytes, offset) exporting this pool's buffer to other processes."""
+        return _wf.wf_ipc_get_mem_handle(self.mem.data_ptr())
+
+    def stall_next_attention(self, key_tile: int, wait_limit_cycles: int) -> None:
+        """Test hook: the next attention launch skips one K load and gives up on
+        its waits after wait_limit_cycles (wf_pool_debug_stall_next_attention)."""
+        st = _wf.wf_pool_debug_stall_next_attention(self.handle, key_tile, wait_limit_cycles)
+        if st != _wf.WF_OK:
+            raise WfError(st, "wf_pool_debug_stall_next_attention")
 
     def advance(self, stream=None) -> None:
         s = 0 if self.device is None else _stream(self.device, stream)

@@ -36,6 +36,8 @@ EXPORTS = (
     "wf_advance_round", "wf_pool_check_status", "wf_pool_destroy", "wf_status_string",
     "wf_pool_round", "wf_pool_get_geometry", "wf_pool_get_layout", "wf_pool_debug_poke_page",
     "wf_project_publish", "wf_publish_kv_slot", "wf_round_attention_slot", "wf_deliver_kv",
+    "wf_pool_debug_stall_next_attention", "wf_ipc_get_mem_handle", "wf_ipc_open_mem",
+    "wf_ipc_close_mem",
 )
 
 
@@ -61,6 +63,10 @@ class WfPoolGeometry(ctypes.Structure):
         ("page_bytes", ctypes.c_size_t), ("total_bytes", ctypes.c_size_t),
         ("kv_scale_offset", ctypes.c_size_t), ("q_scale_offset", ctypes.c_size_t),
     ]
+
+
+class WfIpcHandle(ctypes.Structure):
+    _fields_ = [("bytes", ctypes.c_ubyte * 64)]
 
 
 class WfError(RuntimeError):
@@ -95,7 +101,11 @@ def _load():
         "wf_project_publish": (I32, [P, I32, P, P, P, P]),
         "wf_publish_kv_slot": (I32, [P, I32, I32, P, P, P, P, P]),
         "wf_round_attention_slot": (I32, [P, I32, I32, P, P, P]),
-        "wf_deliver_kv": (I32, [P, I32, I32, P, P]),
+        "wf_deliver_kv": (I32, [P, I32, I32, P, SZ, P]),
+        "wf_pool_debug_stall_next_attention": (I32, [P, I32, I64]),
+        "wf_ipc_get_mem_handle": (I32, [P, ctypes.POINTER(WfIpcHandle), ctypes.POINTER(SZ)]),
+        "wf_ipc_open_mem": (I32, [ctypes.POINTER(WfIpcHandle), SZ, ctypes.POINTER(P)]),
+        "wf_ipc_close_mem": (I32, [P, SZ]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -158,8 +168,41 @@ def wf_round_attention_slot(pool: int, layer: int, slot: int, q_rot: int, out: i
                                         ctypes.c_void_p(stream or None))
 
 
-def wf_deliver_kv(pool: int, layer: int, slot: int, dst_pool_mem: int, stream: int) -> int:
-    return _lib.wf_deliver_kv(pool, layer, slot, dst_pool_mem, ctypes.c_void_p(stream or None))
+def wf_deliver_kv(pool: int, layer: int, slot: int, dst_pool_mem: int, dst_pool_bytes: int,
+                  stream: int) -> int:
+    return _lib.wf_deliver_kv(pool, layer, slot, dst_pool_mem, dst_pool_bytes,
+                              ctypes.c_void_p(stream or None))
+
+
+def wf_pool_debug_stall_next_attention(pool: int, key_tile: int, wait_limit_cycles: int) -> int:
+    return _lib.wf_pool_debug_stall_next_attention(pool, key_tile, wait_limit_cycles)
+
+
+def wf_ipc_get_mem_handle(dev_ptr: int):
+    """(64 handle bytes, offset of dev_ptr inside its allocation)."""
+    h = WfIpcHandle()
+    off = ctypes.c_size_t(0)
+    st = _lib.wf_ipc_get_mem_handle(dev_ptr, ctypes.byref(h), ctypes.byref(off))
+    if st != WF_OK:
+        raise WfError(st, "wf_ipc_get_mem_handle")
+    return bytes(h.bytes), off.value
+
+
+def wf_ipc_open_mem(handle: bytes, offset: int) -> int:
+    """Device pointer of another process's exported buffer, mapped here."""
+    if len(handle) != 64:
+        raise ValueError("an IPC handle is 64 bytes")
+    h = WfIpcHandle()
+    ctypes.memmove(h.bytes, handle, 64)
+    ptr = ctypes.c_void_p(0)
+    st = _lib.wf_ipc_open_mem(ctypes.byref(h), offset, ctypes.byref(ptr))
+    if st != WF_OK:
+        raise WfError(st, "wf_ipc_open_mem")
+    return ptr.value
+
+
+def wf_ipc_close_mem(dev_ptr: int, offset: int) -> int:
+    return _lib.wf_ipc_close_mem(dev_ptr, offset)
 
 
 def wf_advance_round(pool: int, stream: int) -> int:

@@ -192,6 +192,15 @@ wf_status wf_round_attention(wf_pool *pool, int32_t layer, const void *q_rot, vo
  * under WF_MASK_RF, and every rank for the store (its chunk becomes anchor or
  * history for all later rounds). wave_plan() in the Python binding lists them.
  *
+ * Ordering across rounds is the caller's too: a delivery of round k + 1
+ * overwrites the receiver's pages of the same slot (and the recycled store
+ * pages), so a sender must not deliver round k + 1 into a receiver until that
+ * receiver's round-k wf_round_attention_slot has finished reading them (for
+ * example an event the receiver records after its attention, or a barrier
+ * between rounds). The readiness check reads the tags once, when the
+ * attention kernel starts, so it cannot catch an overwrite that lands while
+ * the kernel runs; the output would then be silently wrong.
+ *
  * wf_publish_kv_slot: wf_publish_kv restricted to one live slot: reads only
  * that slot's rows of q, k, v ([S+1][C][heads][d] buffers), writes its q_rot
  * rows, its pages and their ready tags. WF_ERR_CALL_ORDER if the slot is not
@@ -211,21 +220,52 @@ wf_status wf_round_attention_slot(wf_pool *pool, int32_t layer, int32_t slot, co
  * pools, its block scale) is copied to the same physical page of the
  * receiver, then the receiver's ready tags of those pages are set to the
  * slot's tag of this round.
- *   dst_pool_mem : the receiver pool's device buffer (as passed to its
- *                  wf_kv_pool_create), 256-byte aligned and addressable from
- *                  the current device: a buffer on this device or a peer
- *                  device's buffer with peer access enabled (the copy stores
- *                  go over NVLink). The receiver must have this pool's config,
- *                  page order and round (not checked: the receiver may be on
- *                  another process's device).
- * The kernels first check this pool's page ids and ready tags for the slot: a
- * bad id records WF_ERR_BAD_PAGE, a tag from another round WF_ERR_NOT_READY
- * (the slot was not published in this round), in this pool's status word, and
- * nothing is written to the receiver. The tags are written by a second kernel
- * in stream order after the data. WF_ERR_CALL_ORDER if the slot is not live;
+ *   dst_pool_mem   : the receiver pool's device buffer (as passed to its
+ *                    wf_kv_pool_create), 256-byte aligned and addressable from
+ *                    the current device: a buffer on this device, a peer
+ *                    device's buffer with peer access enabled, or a buffer of
+ *                    another process opened with wf_ipc_open_mem (the copy
+ *                    stores go over NVLink when it is on another GPU).
+ *   dst_pool_bytes : the receiver's pool size; WF_ERR_INVALID_ARG unless it
+ *                    equals this pool's wf_kv_pool_bytes.
+ * The receiver must have this pool's config, page order and round. Every pool
+ * stores a 64-bit signature of its config and page order in its memory at
+ * creation; the kernels compare the receiver's with this pool's and, if they
+ * differ, record WF_ERR_INVALID_ARG in this pool's status word and write
+ * nothing. Each copy CTA then checks its own page in this pool: an id out of
+ * range records WF_ERR_BAD_PAGE, a ready tag from another round
+ * WF_ERR_NOT_READY (the slot was not published in this round), and that
+ * page's tiles are not copied. The tag kernel, in stream order after the
+ * copy, checks every page of the slot the same way and stamps the receiver's
+ * tags only if all pass, so the receiver never sees a ready tag for a slot
+ * that was not wholly published and copied; a slot not published at all
+ * leaves the receiver untouched. WF_ERR_CALL_ORDER if the slot is not live;
  * WF_ERR_INVALID_ARG for a NULL, misaligned or self receiver buffer. */
 wf_status wf_deliver_kv(const wf_pool *pool, int32_t layer, int32_t slot, void *dst_pool_mem,
-                        wf_stream_t stream);
+                        size_t dst_pool_bytes, wf_stream_t stream);
+
+/* Inter-process access to a pool buffer, for Wave Parallelism with one
+ * process per stage GPU (Method section and Figure 3c: each stage writes its
+ * K/V straight into the ordered slots of the stages that read it).
+ *
+ * wf_ipc_get_mem_handle: export the device allocation that holds dev_ptr
+ * (a receiver's pool buffer, on the current device) as an opaque handle that
+ * another process can open, plus dev_ptr's byte offset inside that
+ * allocation. WF_ERR_INVALID_ARG if dev_ptr is not device memory of this
+ * process, WF_ERR_CUDA if CUDA refuses the export.
+ * wf_ipc_open_mem: map an exported allocation into this process (on the
+ * current device; peer access to the owner's device is enabled on demand) and
+ * return the pointer at `offset` inside it, to pass to wf_deliver_kv as
+ * dst_pool_mem. WF_ERR_CUDA if the handle cannot be opened (a handle cannot
+ * be opened by the process that exported it).
+ * wf_ipc_close_mem: unmap a pointer returned by wf_ipc_open_mem (same
+ * offset). The exporting process keeps ownership of the memory and must keep
+ * it allocated until every importer has closed it. None of these calls
+ * allocates device memory. */
+typedef struct { unsigned char bytes[64]; } wf_ipc_handle;
+wf_status wf_ipc_get_mem_handle(const void *dev_ptr, wf_ipc_handle *handle, size_t *offset);
+wf_status wf_ipc_open_mem(const wf_ipc_handle *handle, size_t offset, void **dev_ptr);
+wf_status wf_ipc_close_mem(void *dev_ptr, size_t offset);
 
 /* Fused QKV projection + publication for one layer (Method section: the local
  * QKV projection runs without waiting for remote K/V, and K/V are published
@@ -283,6 +323,22 @@ wf_status wf_pool_get_layout(const wf_pool *pool, int32_t *n_positions, int32_t 
  * page ids and record WF_ERR_BAD_PAGE instead of accessing memory. */
 wf_status wf_pool_debug_poke_page(wf_pool *pool, int32_t position, int32_t j,
                                   int32_t physical, wf_stream_t stream);
+
+/* Test hook for the bounded waits of the tensor-core attention kernel
+ * (readiness is checked just before attention, Method section; a kernel whose
+ * wait for a copy or an MMA runs out gives up instead of spinning): the NEXT
+ * wf_round_attention / wf_round_attention_slot call on this pool issues no
+ * load of K for key tile `key_tile` of any query tile (key tiles count the
+ * 128-token pages of the slot's context in order, from 0), so the waits for it
+ * can only run out, and every bounded wait of that launch gives up after
+ * `wait_limit_cycles` SM clock cycles (1000 .. 2e9; the default is 2e9, about
+ * a second). The waits that drain a CTA's own in-flight copies and MMAs keep
+ * their fixed, longer bound. A CTA that gives up records WF_ERR_TIMEOUT,
+ * writes none of its output rows, and frees its tensor memory; CTAs whose
+ * context is shorter than key_tile + 1 tiles run normally. Later launches are
+ * unaffected. bf16 and FP8_E4M3 pools only (WF_ERR_UNSUPPORTED for fp32). */
+wf_status wf_pool_debug_stall_next_attention(wf_pool *pool, int32_t key_tile,
+                                             int64_t wait_limit_cycles);
 
 #ifdef __cplusplus
 }

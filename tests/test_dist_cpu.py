@@ -55,3 +55,30 @@ def test_reference_arm_runs_the_oracle_on_cpu():
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_bench_spawns_its_own_ranks():
+    # `bench.py --gpus 2` outside torchrun relaunches itself as two ranks; the
+    # reference arm then runs on rank 0 only (gloo on a host without GPUs) and
+    # prints one line that reports the world size it ran under.
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--gpus", "2", "--steps", "1", "--warmup", "1",
+                          "--ref-step-seconds", "0.2"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT, env=env)
+    assert out.returncode == 0, out.stderr[-3000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+
+
+def test_peak_follows_observed_conditions():
+    import bench
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    capped = {"reasons": ["sw_power_cap"]}
+    assert bench.pick_peak(peaks, 5.0, capped) == (1400.0, "sustained")
+    assert bench.pick_peak(peaks, 0.5, capped) == (1600.0, "burst")      # too short
+    assert bench.pick_peak(peaks, 5.0, {"reasons": []}) == (1600.0, "burst")
+    assert bench.pick_peak(peaks, 5.0, None) == (1600.0, "burst")

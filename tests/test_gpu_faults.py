@@ -4,14 +4,23 @@ The readiness check of the Method section (K/V must be published before
 attention reads them) and the page bounds checks are exercised by planting the
 error on the host side: a skipped publish leaves stale ready tags, and a test
 hook writes an out-of-range id into the device page table. The kernels record
-the error in the pool's status word and write nothing; no kernel traps,
-faults or waits on a flag that is never set."""
+the error in the pool's status word and write nothing; no kernel traps or
+faults.
+
+The bounded waits of the tensor-core attention kernel are exercised the same
+way: a test hook makes the next launch skip one K load, so the waits for that
+tile can only run out, and shortens their limit to about 0.1 ms. Every CTA
+whose context reaches that tile must record WF_ERR_TIMEOUT, drain its
+in-flight copies and MMAs, free its tensor memory and write no output; CTAs
+with shorter contexts finish normally; and the next launch on the same pool
+must produce the same output as a launch before the stall."""
 import numpy as np
 import pytest
 import torch
 
 import wf_inputs
 import chunk_causal_wavefront_b200 as wfb
+from test_gpu_fp8 import Fp8Rollout
 from wf_test_utils import Rollout
 
 pytestmark = pytest.mark.gpu
@@ -115,3 +124,61 @@ def test_pool_memory_too_small_or_misaligned():
     with pytest.raises(W.WfError) as e:
         W.wf_kv_pool_create(c, mem.data_ptr() + 16, n, None, s)
     assert e.value.status == W.WF_ERR_INVALID_ARG
+
+
+STALL_LIMIT = 200_000   # SM cycles: ~0.1 ms at 1.9 GHz
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("key_tile", [0, 5, 13])
+def test_bounded_wait_runs_out(dtype, key_tile):
+    # CFG: 3 pages per chunk; in a steady round the store reads 4 chunks (12
+    # key tiles) and the denoising slots 5..7 chunks (15..21 tiles). Tile 0
+    # stalls every CTA before its first MMA, tile 5 every CTA mid-stream with
+    # copies and MMAs in flight, tile 13 every CTA except the store's.
+    cfg = CFG.replace(rounds=8)
+    ro = Fp8Rollout(cfg, page_seed=3) if dtype == "fp8" else Rollout(cfg, page_seed=3)
+    for _ in range(cfg.steady_round()):
+        ro.publish(0)
+        ro.pool.advance()
+    ro.publish(0)
+    ro.attention(0)
+    assert ro.pool.check_status() == wfb.WF_OK
+    clean = ro.out.clone()
+    lay = ro.pool.layout()
+    tiles = {slot: (i + 1) * 3 for i, (kind, chunk, slot, tag, pgs) in enumerate(lay)
+             if slot is not None}
+    assert min(tiles.values()) == 12 and max(tiles.values()) == 21
+
+    ro.pool.stall_next_attention(key_tile, STALL_LIMIT)
+    ro.attention(0)                                       # fills out with NaN first
+    assert ro.pool.check_status() == wfb.WF_ERR_TIMEOUT
+    out = ro.out.float()
+    for slot, n in tiles.items():
+        if n > key_tile:
+            assert torch.isnan(out[slot]).all(), (slot, n)   # gave up: nothing written
+        else:
+            assert torch.equal(ro.out[slot].view(torch.int16), clean[slot].view(torch.int16))
+    assert ro.pool.check_status() == wfb.WF_OK            # status cleared after reading
+
+    ro.attention(0)                                       # the hook lasted one launch
+    assert ro.pool.check_status() == wfb.WF_OK
+    for slot in tiles:
+        assert torch.equal(ro.out[slot].view(torch.int16), clean[slot].view(torch.int16)), slot
+    ro.close()
+
+
+def test_stall_hook_arguments():
+    ro = Rollout(CFG, page_seed=1)
+    with pytest.raises(wfb.WfError) as e:
+        ro.pool.stall_next_attention(-1, STALL_LIMIT)
+    assert e.value.status == wfb.WF_ERR_INVALID_ARG
+    with pytest.raises(wfb.WfError) as e:
+        ro.pool.stall_next_attention(0, 10)               # below the minimum limit
+    assert e.value.status == wfb.WF_ERR_INVALID_ARG
+    ro.close()
+    f32 = Rollout(wf_inputs.CONFIGS["tiny_f32"], page_seed=1)
+    with pytest.raises(wfb.WfError) as e:
+        f32.pool.stall_next_attention(0, STALL_LIMIT)
+    assert e.value.status == wfb.WF_ERR_UNSUPPORTED
+    f32.close()

@@ -229,6 +229,28 @@ def test_fp8_full_size_sampled(name):
     assert rec
 
 
+def test_fp8_long_context_past_page_cache():
+    # 29 chunks x 37 pages = 1073 key tiles: page ids and K/V scale exponents
+    # past the 1024 cached in shared memory are read through the page table.
+    cfg = wf_inputs.CONFIGS["wan13b_bf16"].replace(
+        name="long_context_bf16", num_stages=1, num_heads=1, history_chunks=26, rounds=30)
+    positions = cfg.anchor_chunks + cfg.history_chunks + cfg.num_stages + 1
+    assert positions * cfg.pages_per_chunk > 1024
+    ro = Fp8Rollout(cfg, page_seed=6)
+    rows = np.array([0, 1, 127, 128, 777, 2345, 3000, 4607, 4608, 4679])
+    rec = []
+    for k in range(cfg.steady_round() + 1):
+        ro.publish()
+        if k == cfg.steady_round():
+            ro.attention()
+            assert ro.pool.check_status() == 0
+            ro.check_publish()
+            ro.check_attention(rows=rows, record=rec)
+        ro.pool.advance()
+    ro.close()
+    assert rec
+
+
 def test_fp8_value_ones_and_mask_perturbation():
     """V = 1 everywhere gives out = 1 up to the P rounding bound; changing the
     K/V of a noisier slot leaves every cleaner slot's output bit-identical."""

@@ -9,6 +9,7 @@ No rank receives a slot it does not read (except the store's chunk, which
 every rank keeps for later rounds). The multi-process test runs the plan on
 gloo ranks (one per slot), each computing its own sends, and checks that the
 gathered sends are exactly what every rank needs."""
+import ctypes
 import os
 import sys
 
@@ -158,10 +159,28 @@ def test_wave_calls_on_host_only_pools():
     assert W.wf_publish_kv_slot(pool.handle, 0, -1, 16, 16, 16, 32, 0) == W.WF_ERR_INVALID_ARG
     assert W.wf_round_attention_slot(pool.handle, 0, 0, 16, 32, 0) == W.WF_ERR_CALL_ORDER
     assert W.wf_round_attention_slot(pool.handle, 0, -1, 16, 32, 0) == W.WF_ERR_INVALID_ARG
-    assert W.wf_deliver_kv(pool.handle, 0, 0, 256, 0) == W.WF_ERR_CALL_ORDER
-    assert W.wf_deliver_kv(pool.handle, 0, 0, None, 0) == W.WF_ERR_INVALID_ARG
-    assert W.lib().wf_deliver_kv(None, 0, 0, None, None) == W.WF_ERR_INVALID_ARG
+    assert W.wf_deliver_kv(pool.handle, 0, 0, 256, pool.nbytes, 0) == W.WF_ERR_CALL_ORDER
+    assert W.wf_deliver_kv(pool.handle, 0, 0, None, pool.nbytes, 0) == W.WF_ERR_INVALID_ARG
+    assert W.lib().wf_deliver_kv(None, 0, 0, None, 0, None) == W.WF_ERR_INVALID_ARG
+    # the stall hook needs a device pool with a tensor-core attention path
+    assert W.wf_pool_debug_stall_next_attention(pool.handle, 0, 10**6) == W.WF_ERR_CALL_ORDER
+    assert W.lib().wf_pool_debug_stall_next_attention(None, 0, 10**6) == W.WF_ERR_INVALID_ARG
     pool.close()
+
+
+def test_ipc_calls_reject_bad_arguments():
+    # Argument checks only: no CUDA context is needed to refuse these.
+    from chunk_causal_wavefront_b200 import wf as W
+    h = W.WfIpcHandle()
+    off = ctypes.c_size_t(0)
+    ptr = ctypes.c_void_p(0)
+    assert W.lib().wf_ipc_get_mem_handle(None, ctypes.byref(h), ctypes.byref(off)) == W.WF_ERR_INVALID_ARG
+    assert W.lib().wf_ipc_get_mem_handle(256, None, ctypes.byref(off)) == W.WF_ERR_INVALID_ARG
+    assert W.lib().wf_ipc_open_mem(None, 0, ctypes.byref(ptr)) == W.WF_ERR_INVALID_ARG
+    assert W.lib().wf_ipc_open_mem(ctypes.byref(h), 0, None) == W.WF_ERR_INVALID_ARG
+    assert W.lib().wf_ipc_close_mem(None, 0) == W.WF_ERR_INVALID_ARG
+    with pytest.raises(ValueError):
+        W.wf_ipc_open_mem(b"short", 0)
 
 
 def _rank_tables(rank, world, port, q):
