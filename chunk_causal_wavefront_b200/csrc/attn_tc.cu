@@ -105,7 +105,7 @@ struct Fmt {
   static constexpr uint32_t kOffBar = kF8 ? kOffStage + 2 * 32768 : kOffStage;
   static constexpr float kLazy = kF8 ? 4.0f : 8.0f;             // rescale threshold (log2)
   static constexpr int kPShift = 4;                             // E4M3 headroom of P'
-  static constexpr int kNumBars = 24;
+  static constexpr int kNumBars = 26;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // TMEM base, abort, 12 ints
   static constexpr uint32_t kOffPages = kOffMisc + 64;
   static constexpr uint32_t kOffExps = kOffPages + kPageCache * 4;   // int16 ek, ev (FP8)
@@ -116,7 +116,8 @@ constexpr int kNumBars = Fmt<false>::kNumBars;
 enum Bar {
   kQFull = 0, kKFull0 = 1, kKEmpty0 = 3, kVFull0 = 5, kVEmpty0 = 7,
   kSFull0 = 9, kPReady0 = 11, kPVDone0 = 13, kDrain = 15,
-  kTurn0 = 16, kTurn1 = 20   // E4M3: exponential-phase turns, one per sub-partition and tile
+  kTurn0 = 16, kTurn1 = 20,  // E4M3: exponential-phase turns, one per sub-partition and tile
+  kSRead0 = 24               // E4M3: the softmax has read S_q into registers (one per tile)
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -129,8 +130,12 @@ __device__ __forceinline__ float ex2(float x) {
 #define WF_F8_POLY_PAIRS 6
 #endif
 #ifndef WF_F8_TURNS
-#define WF_F8_TURNS 1
+#define WF_F8_TURNS 0
 #endif
+#ifndef WF_BF16_POLY_PAIRS
+#define WF_BF16_POLY_PAIRS 4
+#endif
+constexpr int kBf16PolyPairs = WF_BF16_POLY_PAIRS;
 // E4M3: of every 16 pairs of exponentials, this many run as a polynomial on
 // the FMA pipe instead of the MUFU unit (which does 16 exponentials per clock
 // per SM, in the f32 form as in the packed f16x2/bf16x2 forms: measured).
@@ -141,26 +146,47 @@ constexpr bool kF8Turns = WF_F8_TURNS != 0;
 // and subtracting 1.5 * 2^23 rounds to an integer) and f in [-1/2, 1/2]; 2^f
 // from a degree-2 polynomial whose coefficients minimise the largest relative
 // error on [-1/2, 1/2] (1.73e-3, far below E4M3's half unit of 2^-4); n is
-// added to the exponent field. x is clamped below at -127 first, so -inf
-// (masked keys) and very small probabilities come out as 2^-127 or less,
-// which rounds to zero in E4M3 at any block scale the kernel uses.
+// added to the exponent field. x is clamped below at -126 first, so -inf
+// (masked keys) and very small probabilities come out below 2^-125 (n >= -126
+// keeps the exponent field from borrowing into the sign bit even when
+// 2^f < 1), which rounds to zero in E4M3 at any block scale the kernel uses.
 __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
   float a, b;
   unf2(x2, a, b);
-  const uint64_t xc = f2(fmaxf(a, -127.0f), fmaxf(b, -127.0f));
+  const uint64_t xc = f2(fmaxf(a, -126.0f), fmaxf(b, -126.0f));
   const uint64_t t = fadd2(xc, f2(12582912.0f, 12582912.0f));    // 1.5 * 2^23 + n
   float t0, t1;
   unf2(t, t0, t1);
   const uint64_t nf = fadd2(t, f2(-12582912.0f, -12582912.0f));  // n
-  float n0, n1;
-  unf2(nf, n0, n1);
-  const uint64_t fr = fadd2(xc, f2(-n0, -n1));                    // f
+  const uint64_t fr = ffma2(nf, f2(-1.0f, -1.0f), xc);            // f = x - n, exact
   uint64_t p = ffma2(fr, f2(0.23842734f, 0.23842734f), f2(0.70344603f, 0.70344603f));
   p = ffma2(p, fr, f2(1.0004431f, 1.0004431f));
   float p0, p1;
   unf2(p, p0, p1);
   // the low bits of t's pattern hold n (two's complement); shifted into the
   // exponent field they scale p by 2^n
+  p0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+  return f2(p0, p1);
+}
+
+// The same with a degree-3 polynomial (largest relative error 7.5e-5 on
+// [-1/2, 1/2], far below bf16's half unit of 2^-9), for bf16 P; clamped
+// inputs give less than 2^-125, nothing next to a row sum of at least 1.
+__device__ __forceinline__ uint64_t exp2_poly3(uint64_t x2) {
+  float a, b;
+  unf2(x2, a, b);
+  const uint64_t xc = f2(fmaxf(a, -126.0f), fmaxf(b, -126.0f));
+  const uint64_t t = fadd2(xc, f2(12582912.0f, 12582912.0f));
+  float t0, t1;
+  unf2(t, t0, t1);
+  const uint64_t nf = fadd2(t, f2(-12582912.0f, -12582912.0f));
+  const uint64_t fr = ffma2(nf, f2(-1.0f, -1.0f), xc);
+  uint64_t p = ffma2(fr, f2(0.0551715f, 0.0551715f), f2(0.24261096f, 0.24261096f));
+  p = ffma2(p, fr, f2(0.69326097f, 0.69326097f));
+  p = ffma2(p, fr, f2(0.99992806f, 0.99992806f));
+  float p0, p1;
+  unf2(p, p0, p1);
   p0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
   p1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
   return f2(p0, p1);
@@ -232,6 +258,17 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
   }
 }
 
+// O_q (+)= P_q V(stage) with P_q in shared memory (E4M3: one 128-byte-swizzled
+// [128 rows][128 keys] block, K-major like Q), V MN-major as above.
+__device__ __forceinline__ void issue_pv_f8_smem(uint32_t tmem_o, uint32_t p_lo, uint32_t v_lo,
+                                                 uint32_t hi, bool accumulate_first) {
+  constexpr uint32_t idPV = make_idesc_e4m3(kBM, kHD, true);
+#pragma unroll
+  for (int k = 0; k < kBN / 32; ++k)
+    mma_f8_ss2(tmem_o, p_lo + ((k * 32) >> 4), v_lo + ((k * 4096) >> 4), hi, idPV,
+               (accumulate_first || k > 0) ? 1u : 0u);
+}
+
 template <bool kF8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tq,
@@ -299,8 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
       *abort_flag = 0;
       for (int b = 0; b < kNumBars; ++b) {
-        // p_ready: one elected arrival per softmax warp of the tile
-        const bool softmax_arrives = b == kPReady0 || b == kPReady0 + 1;
+        // p_ready, s_read: one elected arrival per softmax warp of the tile
+        const bool softmax_arrives = b == kPReady0 || b == kPReady0 + 1 || b == kSRead0 ||
+                                     b == kSRead0 + 1;
         mbar_init(bars + b, softmax_arrives ? kBM / 32 : 1);
       }
       fence_barrier_init();
@@ -400,7 +438,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(bars + kKEmpty0);
       }
-      for (int j = 0; ok && j < n_tiles; ++j) {
+      // E4M3: P_q lives in shared memory (in the tile's output staging buffer),
+      // so S_q(j+1) may overwrite S_q(j) in TMEM as soon as the softmax has read
+      // it; the next S is computed while the softmax works on this one, and
+      // only P_q V(j) waits for P_q(j).
+      const uint32_t p_lo = desc_lo_sw128(smem_u32(smem + F::kOffStage), 16);
+      constexpr uint32_t kPStep = 32768 >> 4;                 // tile 1's P (staging) buffer
+      for (int j = 0; kF8 && ok && j < n_tiles; ++j) {
+        const int stg = j & 1, nstg = (j + 1) & 1;
+        if (j + 1 < n_tiles) {
+          if (!wait_bar(ctx, kKFull0 + nstg, ((j + 1) >> 1) & 1)) break;
+          if (!wait_bar(ctx, kSRead0, j & 1)) break;
+          tc_fence_after();
+          issue_s<kF8>(tmem + kTmemS, q_lo, k_lo + nstg * kTileStep, hi);
+          mma_commit(bars + kSFull0);
+          if (has_q1) {
+            if (!wait_bar(ctx, kSRead0 + 1, j & 1)) break;
+            tc_fence_after();
+            issue_s<kF8>(tmem + kTmemS + 128, q_lo + kTileStep, k_lo + nstg * kTileStep, hi);
+            mma_commit(bars + kSFull0 + 1);
+          }
+          mma_commit(bars + kKEmpty0 + nstg);
+        }
+        if (!wait_bar(ctx, kVFull0 + stg, (j >> 1) & 1)) break;
+        if (!wait_bar(ctx, kPReady0, j & 1)) break;
+        tc_fence_after();
+        issue_pv_f8_smem(tmem + kTmemO, p_lo, v_lo + stg * kTileStep, hi, j > 0);
+        mma_commit(bars + kPVDone0);
+        if (has_q1) {
+          if (!wait_bar(ctx, kPReady0 + 1, j & 1)) break;
+          tc_fence_after();
+          issue_pv_f8_smem(tmem + kTmemO + 128, p_lo + kPStep, v_lo + stg * kTileStep, hi, j > 0);
+          mma_commit(bars + kPVDone0 + 1);
+        }
+        mma_commit(bars + kVEmpty0 + stg);
+      }
+      for (int j = 0; !kF8 && ok && j < n_tiles; ++j) {
         const int stg = j & 1, nstg = (j + 1) & 1;
         const bool more = j + 1 < n_tiles;
         if (!wait_bar(ctx, kVFull0 + stg, (j >> 1) & 1)) break;
@@ -480,6 +553,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence32(s + c * 32);
+      if constexpr (kF8) {
+        // S_q is in registers: the issuer may compute the next S_q over it.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + kSRead0 + q);
+      }
 
       if (valid < kBN) {
 #pragma unroll
@@ -513,6 +592,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                               q == 0 ? ((j - 1) & 1) : (j & 1)));
         if (!ok) break;
       }
+      if (kF8 && j > 0) {
+        // P_q(j-1) in shared memory is read by P*V(j-1) until that completes.
+        ok = __all_sync(0xffffffffu, wait_bar(ctx, kPVDone0 + q, (j - 1) & 1));
+        if (!ok) break;
+      }
+      // E4M3: row r of P_q in its 128-byte-swizzled staging block (K-major,
+      // the layout of a Q tile): 16-byte chunk c at r * 128 + (c ^ (r & 7)) * 16.
+      const uint32_t p_row = smem_u32(smem + F::kOffStage + q * 32768 + r * 128);
       const uint64_t sc2 = f2(c_j, c_j), nm2 = f2(dv - m_use, dv - m_use);
       uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -537,7 +624,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c & 1) pw[c >> 1] = join16(half, pr);
             else half = pr;
           }
-          tmem_st8(tS + cc * 8, pw);
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const uint32_t addr = p_row + ((((2 * cc + h2) ^ (r & 7)) & 7) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pw[4 * h2]),
+                         "r"(pw[4 * h2 + 1]), "r"(pw[4 * h2 + 2]), "r"(pw[4 * h2 + 3])
+                         : "memory");
+          }
           if (kF8Turns && cc == 2 && has_q1 && lane == 0)
             mbar_arrive(bars + (q == 0 ? kTurn1 : kTurn0) + (warp & 3));
         } else {
@@ -546,9 +639,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 16; ++c) {
             const int k0 = cc * 32 + 2 * c;
             const uint64_t x2 = ffma2(f2(__uint_as_float(s[k0]), __uint_as_float(s[k0 + 1])), sc2, nm2);
-            float a, b;
-            unf2(x2, a, b);
-            const float e0 = ex2(a), e1 = ex2(b);
+            float e0, e1;
+            if (c % 8 >= 8 - kBf16PolyPairs / 2 - (c < 8 ? kBf16PolyPairs % 2 : 0)) {
+              unf2(exp2_poly3(x2), e0, e1);
+            } else {
+              float a, b;
+              unf2(x2, a, b);
+              e0 = ex2(a);
+              e1 = ex2(b);
+            }
             acc[c & 3] = fadd2(acc[c & 3], f2(e0, e1));
             pw[c] = pack_bf16(e0, e1);
           }
@@ -581,6 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tmem_st_wait();
+      if (kF8) fence_proxy_async_smem();   // P_q's shared-memory stores, read by the MMA
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + kPReady0 + q);

@@ -181,18 +181,6 @@ bool encode_plain_bf16_map(CUtensorMap *map, void *base, int rank, const cuuint6
   return r == CUDA_SUCCESS;
 }
 
-// Unswizzled tiled map over bytes (E4M3 codes).
-bool encode_plain_u8_map(CUtensorMap *map, void *base, int rank, const cuuint64_t *dims,
-                         const cuuint64_t *strides_bytes, const cuuint32_t *box) {
-  auto fn = get_encode();
-  if (!fn) return false;
-  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, base, dims, strides_bytes, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 bool encode_bf16_map(CUtensorMap *map, void *base, int rank, const cuuint64_t *dims,
                      const cuuint64_t *strides_bytes, const cuuint32_t *box) {
   return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box);
@@ -526,13 +514,7 @@ wf_status publish_impl(wf_pool *p, int32_t layer, const void *q, const void *k, 
         !encode_plain_bf16_map(&mv, const_cast<void *>(v), 4, dims, strides, box))
       return WF_ERR_CUDA;
     if (c.dtype == WF_DTYPE_FP8_E4M3) {
-      // q_rot codes: [S+1][C][heads][d] bytes, one box = a 128-row tile of one head
-      const cuuint64_t cstr[3] = {static_cast<cuuint64_t>(c.head_dim),
-                                  static_cast<cuuint64_t>(c.head_dim) * c.num_heads,
-                                  static_cast<cuuint64_t>(c.head_dim) * c.num_heads * c.chunk_tokens};
-      CUtensorMap mqr;
-      if (!encode_plain_u8_map(&mqr, q_rot, 4, dims, cstr, box)) return WF_ERR_CUDA;
-      e = launch_publish_fp8(pp, &mq, &mk, &mv, &mqr, cs);
+      e = launch_publish_fp8(pp, &mq, &mk, &mv, cs);
     } else {
       // q_rot as the inputs; the layer's pages as [pages x 2 x heads x P rows][d],
       // box 64 rows.

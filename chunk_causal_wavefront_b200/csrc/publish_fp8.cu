@@ -14,28 +14,20 @@
 //     (no fused multiply-add), so the codes do not depend on compiler
 //     contraction choices.
 //
-// Work unit: one block of one tensor, i.e. (live slot, page j, head, q|k|v):
-// 128 token rows x 128 dims of bf16 in (32 KB), 16 KB of codes and one scale
-// out. q, k and v of a (slot, page, head) are independent units, since each
-// has its own scale. The kernel is persistent, one CTA per SM walking the
-// units blockIdx.x, blockIdx.x + gridDim.x, ... through a six-stage
-// shared-memory ring:
-//   * a TMA warp loads each unit's tile (box 128 dims x 1 head x 128 rows,
-//     rows past C zero-filled); once the unit is quantised it stores the codes
-//     from the same stage: q_rot through a tensor map over the codes (rows
-//     past C clipped), a K or V page block (16 KB, contiguous in the pool) as
-//     one bulk copy; it writes the block's scale, stamps the page's ready tag
-//     (at the K block of head 0) and refills the stage with the unit six steps
-//     ahead once the stores have read it;
+// Work unit: one (live slot, page j, head) block, i.e. 128 token rows x 128
+// dims of q, k and v (96 KB of bf16 in, 48 KB of codes out). The kernel is a
+// persistent streaming loop, one CTA per SM, each walking the blocks
+// blockIdx.x, blockIdx.x + gridDim.x, ...:
+//   * thread 0 loads the next-but-one block's q, k and v tiles with TMA into a
+//     two-stage shared-memory ring (box 128 dims x 1 head x 128 rows, rows past
+//     C zero-filled), so HBM reads of block i+1 overlap the work on block i;
 //   * 512 threads, 16 per row (8 dims = 16 bytes each), 32 rows per pass, 4
-//     passes: the (cos, sin) entries of the thread's rows are loaded before
-//     the wait for the tile; pass 1 rotates q and k in registers and takes the
-//     block maximum (warp max, then one named barrier over the 16 warps);
-//     pass 2 scales by 2^-e, converts to E4M3 and writes the codes in place
-//     over the stage (row r at byte 128 r: every thread has read the tile by
-//     the barrier). Rows past C are +0 in the tile and stay +0 (rotating them
-//     could turn +0 into -0), so the K and V page blocks get zero codes there.
-// HBM-bound: 2 bytes read and 1 written per (token, head, dim) of q, k and v.
+//     passes: pass 1 rotates q and k (kept in registers) and takes the three
+//     block maxima (warp max, then shared memory across the 16 warps); pass 2
+//     scales by 2^-e, converts to E4M3 and writes 8 bytes per row and thread
+//     (q_rot rows < C, and the whole 128-row K and V page blocks, whose rows
+//     past C are zero codes).
+// HBM-bound: 6 bytes read and 3 written per (token, head, dim).
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -49,22 +41,18 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kRows = 128;                              // rows per block (page / query tile)
-constexpr int kComputeThreads = 512;
-constexpr int kComputeWarps = kComputeThreads / 32;     // 16
-constexpr int kThreads = kComputeThreads + 32;          // + the TMA warp
-constexpr int kTPR = 16;                                // threads per row
-constexpr int kRowsPerPass = kComputeThreads / kTPR;    // 32
-constexpr int kPasses = kRows / kRowsPerPass;           // 4
-constexpr uint32_t kTileBytes = kRows * 128 * 2;        // one bf16 tile, 32 KB
-constexpr uint32_t kCodeBytes = kRows * 128;            // its codes, 16 KB
-constexpr int kStages = 6;
-constexpr uint32_t kOffBars = kStages * kTileBytes;     // full[kStages], quantised[kStages]
-constexpr uint32_t kOffExp = kOffBars + 2 * kStages * 8;          // int [kStages]
-constexpr uint32_t kOffRed = kOffExp + kStages * 4;               // uint32 [2][kComputeWarps]
-constexpr uint32_t kOffMisc = kOffRed + 2 * kComputeWarps * 4;    // abort flag
-constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
-enum { kFull0 = 0, kQuant0 = kStages };
+constexpr int kRows = 128;                     // rows per block (page / query tile)
+constexpr int kThreads = 512;
+constexpr int kTPR = 16;                       // threads per row
+constexpr int kRowsPerPass = kThreads / kTPR;  // 32
+constexpr int kPasses = kRows / kRowsPerPass;  // 4
+constexpr int kWarps = kThreads / 32;
+constexpr uint32_t kTensorBytes = kRows * 128 * 2;      // one bf16 tile, 32 KB
+constexpr uint32_t kStageBytes = 3 * kTensorBytes;      // q, k, v
+constexpr uint32_t kOffBars = 2 * kStageBytes;          // two stages
+constexpr uint32_t kOffRed = kOffBars + 64;             // [3][kWarps] block maxima
+constexpr uint32_t kOffPos = kOffRed + 3 * kWarps * 4;  // [kRows][4] rotary table offsets
+constexpr uint32_t kSmemBytes = kOffPos + 4 * kRows * 4 + 1024;
 
 // Smallest e with amax * 2^-e <= 448 = 1.75 * 2^8, clamped below at -100:
 // for amax = f * 2^E (f in [1, 2)), e = E - 8 if f <= 1.75, else E - 7.
@@ -127,152 +115,72 @@ __device__ __forceinline__ uint2 quant8(const float *v, float mul) {
   return w;
 }
 
-struct Unit {
-  int li, j, h, t;   // live slot index, page of the chunk, head, tensor (0 q, 1 k, 2 v)
+struct Block {
+  int li, j, h;
 };
 
-__device__ __forceinline__ Unit decode(int b, const PublishParams &p) {
-  Unit u;
-  u.t = b % 3;
-  const int blk = b / 3;
+__device__ __forceinline__ Block decode(int b, const PublishParams &p) {
+  Block k;
   const int per_slot = p.npc * p.Hh;
-  u.li = blk / per_slot;
-  const int rem = blk - u.li * per_slot;
-  u.j = rem / p.Hh;
-  u.h = rem - u.j * p.Hh;
-  return u;
+  k.li = b / per_slot;
+  const int rem = b - k.li * per_slot;
+  k.j = rem / p.Hh;
+  k.h = rem - k.j * p.Hh;
+  return k;
 }
 
-// Physical page holding page j of a slot's chunk (-1 if the table is bad).
-__device__ __forceinline__ int block_page(const PublishParams &p, int slot, int j) {
-  const int tpos = __ldg(p.table + kTabSlotPos + slot);
-  const int phys = tpos < 0 ? -1 : __ldg(p.table + kTabPages + tpos * p.npc + j);
-  return (phys < 0 || phys >= p.num_pages) ? -1 : phys;
+// Thread 0: the three TMA tile loads of block b into stage buffer `buf`.
+__device__ __forceinline__ void load_block(int b, uint8_t *buf, uint64_t *bar,
+                                           const PublishParams &p, const CUtensorMap *tq,
+                                           const CUtensorMap *tk, const CUtensorMap *tv) {
+  const Block k = decode(b, p);
+  const int slot = p.live.slot[k.li];
+  mbar_arrive_expect_tx(bar, kStageBytes);
+  tma_load_4d(buf, tq, bar, 0, k.h, k.j * kRows, slot);
+  tma_load_4d(buf + kTensorBytes, tk, bar, 0, k.h, k.j * kRows, slot);
+  tma_load_4d(buf + 2 * kTensorBytes, tv, bar, 0, k.h, k.j * kRows, slot);
 }
 
-// The TMA load of unit b's tile into stage buffer `buf`.
-__device__ __forceinline__ void load_unit(int b, uint8_t *buf, uint64_t *bar,
-                                          const PublishParams &p, const CUtensorMap *tq,
-                                          const CUtensorMap *tk, const CUtensorMap *tv) {
-  const Unit u = decode(b, p);
-  const int slot = p.live.slot[u.li];
-  mbar_arrive_expect_tx(bar, kTileBytes);
-  tma_load_4d(buf, u.t == 0 ? tq : (u.t == 1 ? tk : tv), bar, 0, u.h, u.j * kRows, slot);
-}
-
-// Max over the 512 compute threads (named barrier 1) of non-negative floats
-// compared as bit patterns (the same order for every non-negative value, NaN
-// above +inf), the same result in every one of them. `red` holds one value
-// per warp. A thread passes kAbortBits (above every non-negative pattern)
-// when its wait ran out, so that all threads leave at the same unit.
-constexpr uint32_t kAbortBits = 0xFFFFFFFFu;
-
-__device__ __forceinline__ uint32_t compute_max(uint32_t bits, uint32_t *red) {
-  const uint32_t w = __reduce_max_sync(0xffffffffu, bits);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = w;
-  asm volatile("bar.sync 1, %0;" ::"n"(kComputeThreads) : "memory");
-  uint32_t m = red[0];
+// Block-wide maxima of three non-negative values (every thread gets them).
+__device__ __forceinline__ void block_max3(float (&a)[3], float *red) {
+  const int warp = threadIdx.x >> 5;
 #pragma unroll
-  for (int i = 1; i < kComputeWarps; ++i) m = max(m, red[i]);
-  return m;
+  for (int t = 0; t < 3; ++t) {
+    const uint32_t w = __reduce_max_sync(0xffffffffu, __float_as_uint(a[t]));
+    if ((threadIdx.x & 31) == 0) red[t * kWarps + warp] = __uint_as_float(w);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int t = 0; t < 3; ++t) {
+    float m = red[t * kWarps];
+#pragma unroll
+    for (int i = 1; i < kWarps; ++i) m = fmaxf(m, red[t * kWarps + i]);
+    a[t] = m;
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     publish_fp8_kernel(const __grid_constant__ PublishParams p,
                        const __grid_constant__ CUtensorMap tq,
                        const __grid_constant__ CUtensorMap tk,
-                       const __grid_constant__ CUtensorMap tv,
-                       const __grid_constant__ CUtensorMap tqr) {
+                       const __grid_constant__ CUtensorMap tv) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars);
-  volatile int *exps = reinterpret_cast<volatile int *>(smem + kOffExp);
-  uint32_t *red = reinterpret_cast<uint32_t *>(smem + kOffRed);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc);
-  const int nunits = p.live.n * p.npc * p.Hh * 3;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBars);   // [2]
+  float *red = reinterpret_cast<float *>(smem + kOffRed);
+  int32_t *pos = reinterpret_cast<int32_t *>(smem + kOffPos);      // [row][t, h, w, -]
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBars + 16);
+  const int nblk = p.live.n * p.npc * p.Hh;
   const int G = gridDim.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const Ctx ctx{bars, abort_flag, p.status};
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bars + kFull0 + s, 1);
-      mbar_init(bars + kQuant0 + s, kComputeWarps);
-    }
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  __syncthreads();
-
-  if (warp == kComputeWarps) {
-    // ------------------------------------------------------------ TMA warp --
-    if (lane == 0) {
-      tma_prefetch_desc(&tq);
-      tma_prefetch_desc(&tk);
-      tma_prefetch_desc(&tv);
-      tma_prefetch_desc(&tqr);
-      int issued[kStages] = {};
-      for (int s = 0; s < kStages; ++s) {
-        const int b = blockIdx.x + s * G;
-        if (b < nunits) {
-          load_unit(b, smem + s * kTileBytes, bars + kFull0 + s, p, &tq, &tk, &tv);
-          ++issued[s];
-        }
-      }
-      for (int i = 0;; ++i) {
-        const int b = blockIdx.x + i * G;
-        if (b >= nunits) break;
-        const int s = i % kStages;
-        if (!wait_bar(ctx, kQuant0 + s, (i / kStages) & 1)) break;
-        const Unit u = decode(b, p);
-        const int slot = p.live.slot[u.li];
-        const float scale = exp2i(exps[s]);
-        const uint8_t *buf = smem + s * kTileBytes;
-        if (u.t == 0) {
-          tma_store_4d(&tqr, buf, 0, u.h, u.j * kRows, slot);
-          p.q_scale[(static_cast<size_t>(slot) * p.npc + u.j) * p.Hh + u.h] = scale;
-        } else {
-          const int phys = block_page(p, slot, u.j);
-          if (phys >= 0) {
-            const size_t blk = (static_cast<size_t>(phys) * 2 + (u.t - 1)) * p.Hh + u.h;
-            bulk_store(reinterpret_cast<uint8_t *>(p.pages) + blk * kCodeBytes, buf, kCodeBytes);
-            p.kv_scale[blk] = scale;
-            if (u.t == 1 && u.h == 0) p.tags[phys] = p.live.tag[u.li];
-          } else {
-            record_status(p.status, WF_ERR_BAD_PAGE);
-          }
-        }
-        tma_store_commit();
-        // Refill the previous unit's stage once its stores have read it (the
-        // store just issued may still be reading this one).
-        if (i > 0) {
-          const int bp = b - G + kStages * G;
-          if (bp < nunits) {
-            const int sp = (i - 1) % kStages;
-            tma_store_wait_read_but_last();
-            load_unit(bp, smem + sp * kTileBytes, bars + kFull0 + sp, p, &tq, &tk, &tv);
-            ++issued[sp];
-          }
-        }
-      }
-      // Every store has written global memory and every load has landed
-      // before the CTA exits (only an aborted loop leaves loads behind).
-      tma_store_wait_all();
-      for (int s = 0; s < kStages; ++s)
-        if (issued[s]) drain_wait(ctx, kFull0 + s, (issued[s] - 1) & 1);
-    }
-    return;
-  }
-
-  // -------------------------------------------------------- compute warps --
   const int cv = threadIdx.x & (kTPR - 1);        // 16-byte vector of the head row
   const int r0 = threadIdx.x / kTPR;              // first row of this thread
+  const Ctx ctx{full, abort_flag, p.status};
   // Rotary (cos, sin) entries of this thread's 4 pairs (pairs 4 cv .. 4 cv + 3):
-  // pair pr lies in band t, h or w (band index b); its entry for a row is
-  // rope_t[o + q_b], o the pair's offset from the t table (the three tables
-  // share the pool buffer) and q_b the row's position in band b times that
-  // band's pair count. ctab[i] packs 4 o + b.
+  // pair pr lies in band t, h or w (band index b); its entry for row r is
+  // rope_t[o + pos[4 r + b]], o the pair's offset from the t table (the three
+  // tables share the pool buffer) and pos the row's position in each band
+  // times that band's pair count. ctab[i] packs 4 o + b.
   const int h0 = p.split0 >> 1, h1 = p.split1 >> 1, h2 = p.split2 >> 1;
   int ctab[4] = {0, 0, 0, 0};
   if (p.rope) {
@@ -285,86 +193,137 @@ __global__ void __launch_bounds__(kThreads, 1)
       else ctab[i] = 4 * (ow + pr - h0 - h1) + 2;
     }
   }
+
+  if (threadIdx.x == 0) {
+    mbar_init(full, 1);
+    mbar_init(full + 1, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+  }
+  __syncthreads();
+  int issued0 = 0, issued1 = 0;                   // loads issued per stage (thread 0)
+  if (threadIdx.x == 0) {
+    if (static_cast<int>(blockIdx.x) < nblk) {
+      load_block(blockIdx.x, smem, full, p, &tq, &tk, &tv);
+      ++issued0;
+    }
+    if (static_cast<int>(blockIdx.x) + G < nblk) {
+      load_block(blockIdx.x + G, smem + kStageBytes, full + 1, p, &tq, &tk, &tv);
+      ++issued1;
+    }
+  }
+
   for (int i = 0;; ++i) {
     const int b = blockIdx.x + i * G;
-    if (b >= nunits) break;
-    const int s = i % kStages;
-    const Unit u = decode(b, p);
-    const bool rot = p.rope && u.t < 2;
-    // The (cos, sin) entries of this thread's rows are loaded while the tile
-    // is still in flight. Rotary positions are absolute: frame F * chunk +
-    // n / (gh gw), row y, column x.
-    float2 cs[kPasses][4];
-    if (rot) {
-      const int hw = p.gh * p.gw, t0 = p.F * p.live.chunk[u.li];
-#pragma unroll
-      for (int ps = 0; ps < kPasses; ++ps) {
-        int n = u.j * kRows + r0 + ps * kRowsPerPass;
-        if (n >= p.C) n = 0;
-        const int f = n / hw, yx = n - f * hw, y = yx / p.gw;
-        const int pt = (t0 + f) * h0, py = y * h1, px = (yx - y * p.gw) * h2;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int band = ctab[c] & 3;
-          cs[ps][c] = __ldg(p.rope_t + (ctab[c] >> 2) + (band == 0 ? pt : band == 1 ? py : px));
-        }
-      }
+    if (b >= nblk) break;
+    const int stage = i & 1;
+    const Block blk = decode(b, p);
+    const int li = blk.li, j = blk.j, h = blk.h;
+    const int slot = p.live.slot[li];
+    const int tpos = __ldg(p.table + kTabSlotPos + slot);
+    int phys = tpos < 0 ? -1 : __ldg(p.table + kTabPages + tpos * p.npc + j);
+    if (phys >= p.num_pages) phys = -1;
+    if (phys < 0 && threadIdx.x == 0) record_status(p.status, WF_ERR_BAD_PAGE);
+
+    // Rotary positions of the block's rows (absolute: frame F * chunk + n / (gh gw)).
+    if (p.rope && threadIdx.x < kRows) {
+      int n = j * kRows + threadIdx.x;
+      if (n >= p.C) n = 0;
+      const int hw = p.gh * p.gw, f = n / hw, yx = n - f * hw, y = yx / p.gw;
+      pos[4 * threadIdx.x] = (p.F * p.live.chunk[li] + f) * h0;
+      pos[4 * threadIdx.x + 1] = y * h1;
+      pos[4 * threadIdx.x + 2] = (yx - y * p.gw) * h2;
     }
-    // The n-th use of a stage waits for its n-th fill: parity (i / kStages) & 1.
-    const bool ok = __all_sync(0xffffffffu, wait_bar(ctx, kFull0 + s, (i / kStages) & 1));
-    uint8_t *buf = smem + s * kTileBytes;
-    float x[kPasses][8];
-    float amax = 0.0f;
-    if (!ok) {
-      // nothing to read: the tile never arrived
-    } else if (u.t < 2) {
-#pragma unroll
-      for (int ps = 0; ps < kPasses; ++ps) {
-        const int r = r0 + ps * kRowsPerPass;
-        widen(*reinterpret_cast<const uint4 *>(buf + r * 256 + cv * 16), x[ps]);
-        if (rot && u.j * kRows + r < p.C) rotate8(x[ps], cs[ps]);   // rows past C stay +0
-#pragma unroll
-        for (int c = 0; c < 8; c += 2) amax = max3(amax, fabsf(x[ps][c]), fabsf(x[ps][c + 1]));
-      }
-    } else {
-      uint32_t av = 0;
-#pragma unroll
-      for (int ps = 0; ps < kPasses; ++ps) {
-        const uint4 raw = *reinterpret_cast<const uint4 *>(buf + (r0 + ps * kRowsPerPass) * 256 + cv * 16);
-        av = absmax_bf16x8(av, raw);
-        widen(raw, x[ps]);
-      }
-      amax = fmaxf(__uint_as_float(av << 16), __uint_as_float(av & 0xFFFF0000u));
-    }
-    const uint32_t m = compute_max(ok ? __float_as_uint(amax) : kAbortBits,
-                                   red + (i & 1) * kComputeWarps);
-    if (m == kAbortBits) break;
-    const int e = scale_exponent(__uint_as_float(m));
-    const float mul = exp2i(-e);
+    // The n-th use of a stage waits for its n-th fill: parity (i / 2) & 1.
+    const bool ok = __all_sync(0xffffffffu, wait_bar(ctx, stage, (i >> 1) & 1));
+    if (__syncthreads_or(!ok)) break;             // also publishes pos[] to all threads
+
+    const uint8_t *buf = smem + stage * kStageBytes;
+    float xq[kPasses][8], xk[kPasses][8];
+    uint4 rv[kPasses];
+    float aq = 0.0f, ak = 0.0f;
+    uint32_t av = 0;
 #pragma unroll
     for (int ps = 0; ps < kPasses; ++ps) {
       const int r = r0 + ps * kRowsPerPass;
-      const uint2 w = quant8(x[ps], mul);
-      asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(smem_u32(buf + r * 128 + cv * 8)),
-                   "r"(w.x), "r"(w.y)
-                   : "memory");
+      const uint32_t off = r * 256 + cv * 16;
+      widen(*reinterpret_cast<const uint4 *>(buf + off), xq[ps]);
+      widen(*reinterpret_cast<const uint4 *>(buf + kTensorBytes + off), xk[ps]);
+      rv[ps] = *reinterpret_cast<const uint4 *>(buf + 2 * kTensorBytes + off);
+      // rows past C stay +0 (zero codes): rotating them could turn +0 into -0
+      if (p.rope && j * kRows + r < p.C) {
+        float2 cs[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) cs[c] = __ldg(p.rope_t + (ctab[c] >> 2) + pos[4 * r + (ctab[c] & 3)]);
+        rotate8(xq[ps], cs);
+        rotate8(xk[ps], cs);
+      }
+#pragma unroll
+      for (int c = 0; c < 8; c += 2) {
+        aq = max3(aq, fabsf(xq[ps][c]), fabsf(xq[ps][c + 1]));
+        ak = max3(ak, fabsf(xk[ps][c]), fabsf(xk[ps][c + 1]));
+      }
+      av = absmax_bf16x8(av, rv[ps]);
     }
-    if (threadIdx.x == 0) exps[s] = e;
-    // The codes are read by the TMA / bulk stores (async proxy).
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bars + kQuant0 + s);
+    float amax[3] = {aq, ak, fmaxf(__uint_as_float(av << 16), __uint_as_float(av & 0xFFFF0000u))};
+    block_max3(amax, red);
+    // Every thread has read this stage (and red[]): thread 0 refills the stage
+    // with the next-but-one block while the codes below are written.
+    __syncthreads();
+    if (threadIdx.x == 0 && b + 2 * G < nblk) {
+      load_block(b + 2 * G, smem + stage * kStageBytes, full + stage, p, &tq, &tk, &tv);
+      if (stage) ++issued1; else ++issued0;
+    }
+
+    const int eq = scale_exponent(amax[0]), ek = scale_exponent(amax[1]), ev = scale_exponent(amax[2]);
+    const float mq = exp2i(-eq), mk = exp2i(-ek), mv = exp2i(-ev);
+    const size_t slot_off = static_cast<size_t>(slot) * p.C * p.Hh * p.d;
+    uint8_t *qdst = static_cast<uint8_t *>(p.q_rot) + slot_off + static_cast<size_t>(h) * p.d + cv * 8;
+    const size_t kblk = (static_cast<size_t>(phys < 0 ? 0 : phys) * 2) * p.Hh + h;
+    uint8_t *kdst = reinterpret_cast<uint8_t *>(p.pages) + kblk * p.P * p.d + cv * 8;
+    uint8_t *vdst = kdst + static_cast<size_t>(p.Hh) * p.P * p.d;
+    if (threadIdx.x == 0) {
+      p.q_scale[(static_cast<size_t>(slot) * p.npc + j) * p.Hh + h] = exp2i(eq);
+      if (phys >= 0) {
+        p.kv_scale[kblk] = exp2i(ek);
+        p.kv_scale[kblk + p.Hh] = exp2i(ev);
+      }
+    }
+#pragma unroll
+    for (int ps = 0; ps < kPasses; ++ps) {
+      const int r = r0 + ps * kRowsPerPass;
+      const int n = j * kRows + r;
+      if (n < p.C)
+        *reinterpret_cast<uint2 *>(qdst + static_cast<size_t>(n) * p.Hh * p.d) = quant8(xq[ps], mq);
+      if (phys >= 0) {
+        float xv[8];
+        widen(rv[ps], xv);
+        *reinterpret_cast<uint2 *>(kdst + r * p.d) = quant8(xk[ps], mk);
+        *reinterpret_cast<uint2 *>(vdst + r * p.d) = quant8(xv, mv);
+      }
+    }
+    if (phys >= 0 && h == 0 && threadIdx.x == 0) p.tags[phys] = p.live.tag[li];
+  }
+  // Drain: every load thread 0 issued has landed before the CTA exits. Only
+  // an aborted loop leaves loads behind; waiting on the parity of a stage's
+  // last fill returns at once when that fill was already consumed.
+  if (threadIdx.x == 0) {
+    if (issued0) drain_wait(ctx, 0, (issued0 - 1) & 1);
+    if (issued1) drain_wait(ctx, 1, (issued1 - 1) & 1);
   }
 }
 
 }  // namespace
 
 cudaError_t launch_publish_fp8(const PublishParams &p, const void *tmap_q, const void *tmap_k,
-                               const void *tmap_v, const void *tmap_qrot, cudaStream_t st) {
+                               const void *tmap_v, cudaStream_t st) {
   if (p.live.n == 0) return cudaSuccess;
   if (p.d != 128 || p.P != kRows) return cudaErrorInvalidValue;
-  const int64_t nunits = static_cast<int64_t>(p.live.n) * p.npc * p.Hh * 3;
-  if (nunits > 0x7fffffff) return cudaErrorInvalidValue;
+  const int64_t nblk = static_cast<int64_t>(p.live.n) * p.npc * p.Hh;
+  if (nblk > 0x7fffffff) return cudaErrorInvalidValue;
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -372,10 +331,10 @@ cudaError_t launch_publish_fp8(const PublishParams &p, const void *tmap_q, const
   e = cudaFuncSetAttribute(publish_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  const int grid = static_cast<int>(nunits < sms ? nunits : sms);
+  const int grid = static_cast<int>(nblk < sms ? nblk : sms);
   publish_fp8_kernel<<<grid, kThreads, kSmemBytes, st>>>(
       p, *static_cast<const CUtensorMap *>(tmap_q), *static_cast<const CUtensorMap *>(tmap_k),
-      *static_cast<const CUtensorMap *>(tmap_v), *static_cast<const CUtensorMap *>(tmap_qrot));
+      *static_cast<const CUtensorMap *>(tmap_v));
   return cudaGetLastError();
 }
 

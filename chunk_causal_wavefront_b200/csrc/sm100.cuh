@@ -98,14 +98,6 @@ __device__ __forceinline__ void tma_store_2d(const void *desc, const void *src, 
       : "memory");
 }
 
-// Untiled bulk copy of `bytes` (a multiple of 16) from shared memory to global
-// memory; both addresses 16-byte aligned. Completes through the bulk group.
-__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
-               "r"(smem_u32(src)), "r"(bytes)
-               : "memory");
-}
-
 __device__ __forceinline__ void tma_store_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -119,12 +111,6 @@ __device__ __forceinline__ void tma_store_wait_all() {
 // flight).
 __device__ __forceinline__ void tma_store_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
-// Wait until at most the most recently committed bulk group is still reading
-// shared memory (all older groups have finished reading theirs).
-__device__ __forceinline__ void tma_store_wait_read_but_last() {
-  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
 // Make generic-proxy shared-memory writes visible to the async proxy

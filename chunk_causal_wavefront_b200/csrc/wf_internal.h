@@ -108,11 +108,9 @@ constexpr size_t kSignatureOffset = 8;
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_publish_f32(const PublishParams &p, cudaStream_t st);
 // The FP8 publish takes unswizzled tensor maps of q, k and v over
-// [S+1][C][heads][d] bf16 with a box of 128 dims x 1 head x 128 rows, and an
-// unswizzled map of the q_rot codes over [S+1][C][heads][d] bytes with the
-// same box.
+// [S+1][C][heads][d] bf16 with a box of 128 dims x 1 head x 128 rows.
 cudaError_t launch_publish_fp8(const PublishParams &p, const void *tmap_q, const void *tmap_k,
-                               const void *tmap_v, const void *tmap_qrot, cudaStream_t st);
+                               const void *tmap_v, cudaStream_t st);
 // The bf16 publish for d = 128 and 128-token pages takes unswizzled maps of q,
 // k, v and q_rot over [S+1][C][heads][d] bf16 with a box of 128 dims x 1 head x
 // 64 rows, and an unswizzled 2D map over the layer's pool rows

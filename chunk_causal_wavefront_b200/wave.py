@@ -14,7 +14,16 @@ history chunk of every later round, so it goes to every rank, live or not.
 
 The plan is host logic only: each rank computes the same plan from (S, k,
 mask) with no communication, and calls wf_deliver_kv for its own slot's
-entries."""
+entries.
+
+Ordering is the caller's: a receiver may run its round-k attention only after
+every round-k delivery into its pool has landed, and a sender must not deliver
+round k + 1 into a receiver until that receiver's round-k attention has
+finished reading its pages, since the delivery overwrites the same pages (and
+the recycled store pages) in place. A barrier after each round's attention, or
+an event the receiver records after it and the sender waits for, gives that
+order; the readiness check reads the ready tags once, when the attention kernel
+starts, so it cannot catch an overwrite that lands while the kernel runs."""
 from typing import Dict, List
 
 
