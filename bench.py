@@ -607,10 +607,68 @@ def attention_block(att_ms, flops, timed_s, clocks, peaks, ratio):
             "peak": ratio * peak, "peak_basis": basis, "frac": tflops / (ratio * peak)}
 
 
+def run_deliver(local, peaks, launches=50):
+    """wf_deliver_kv of one live slot's K/V (one layer of the 1.3B-shaped
+    workload) into a second pool on the same device: a same-device copy, so it
+    measures the kernels, not the NVLink path the call is for on several GPUs."""
+    import torch
+    import wf_inputs
+    from chunk_causal_wavefront_b200 import KVPool, make_config
+    cfg = wf_inputs.CONFIGS["wan13b_bf16"]
+    dev = torch.device("cuda", local)
+    npages = (cfg.num_stages + 1 + cfg.anchor_chunks + cfg.history_chunks) * cfg.pages_per_chunk
+    steady = cfg.steady_round()
+    pc = make_config(num_stages=cfg.num_stages, chunk_tokens=cfg.chunk_tokens, num_heads=cfg.num_heads,
+                     head_dim=cfg.head_dim, anchor_chunks=cfg.anchor_chunks,
+                     history_chunks=cfg.history_chunks, page_tokens=cfg.page_tokens, num_layers=1,
+                     dtype=cfg.dtype, rope=cfg.rope, frames_per_chunk=cfg.frames_per_chunk,
+                     grid_h=cfg.grid_h, grid_w=cfg.grid_w, rope_split=cfg.rope_split,
+                     rope_base=cfg.rope_base, max_rounds=steady + 2)
+    order = wf_inputs.draw_page_order(npages, cfg.seed + 1)
+    sender = KVPool(pc, device=dev, page_order=order)
+    receiver = KVPool(pc, device=dev, page_order=order)
+    shape = (cfg.num_slots, cfg.chunk_tokens, cfg.num_heads, cfg.head_dim)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(cfg.seed * 1000 + 7)
+    x = [torch.randn(shape, generator=gen, device=dev).to(torch.bfloat16) for _ in range(3)]
+    q_rot = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    for _ in range(steady):
+        sender.advance()
+        receiver.advance()
+    sender.publish(0, x[0], x[1], x[2], q_rot)
+    slot = 0
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(3):
+        sender.deliver(0, slot, receiver)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(launches)]
+    torch.cuda.synchronize()
+    for a, b in ev:
+        a.record(stream)
+        sender.deliver(0, slot, receiver)
+        b.record(stream)
+    torch.cuda.synchronize()
+    if sender.check_status() != 0 or receiver.check_status() != 0:
+        raise RuntimeError("device status after the delivery timing")
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    tiles = cfg.pages_per_chunk * 2 * cfg.num_heads
+    moved = 2 * tiles * cfg.page_tokens * cfg.head_dim * 2        # read + write, bf16
+    sender.close()
+    receiver.close()
+    gbs = moved / (ms * 1e-3) / 1e9
+    return {"kernels": "deliver_copy_kernel + deliver_tags_kernel",
+            "what": f"one live slot's K/V of one layer ({cfg.pages_per_chunk} pages x K,V x "
+                    f"{cfg.num_heads} heads x {cfg.page_tokens}x{cfg.head_dim} bf16) into a second "
+                    "pool on the same device (same-device copy, not the NVLink path)",
+            "ms_per_launch": ms, "bytes_per_launch": moved, "same_device_copy_gbs": gbs,
+            "pct_hbm": 100 * gbs / peaks["hbm_gbs"], "launches": launches}
+
+
 def run_extras(args, ws, rank, local, peaks):
     """The other workloads, measured in the same run: the 14B-shaped layer and
-    the 5-step layer (steady layer-rounds, publish + attention + advance), and
-    the 30-layer streaming rollout (whole rounds from round 0, fill included)."""
+    the 5-step layer (steady layer-rounds, publish + attention + advance), the
+    Wave Parallelism delivery of one slot (same-device copy), and the 30-layer
+    streaming rollout (whole rounds from round 0, fill included)."""
     import argparse as _ap
     extra = {}
     for name in ("wan14b_bf16", "wan13b_5step_bf16"):
@@ -627,6 +685,9 @@ def run_extras(args, ws, rank, local, peaks):
                 "attention": attention_block(r["att_ms"], r["flops"], timed_s, r["clocks"], peaks, 1.0),
                 "publish_gbs": r["pbytes"] / (r["pub_ms"] * 1e-3) / 1e9,
                 "clocks": r["clocks"]}
+    d = run_deliver(local, peaks)
+    if rank == 0:
+        extra["deliver"] = d
     a = _ap.Namespace(**vars(args))
     a.config, a.steps, a.warmup = "stream_13b_bf16", args.stream_rounds, 3
     r = run_stream(a, ws, rank, local)
