@@ -3,7 +3,13 @@ against the oracle of oracle/wf_fp8.py (codes and scales) and oracle/wf_oracle.p
 (attention over the dequantised operands).
 
 Publication is checked bit for bit: every E4M3 code of q_rot and of the K/V
-pages, every block scale, the zero tails and the ready tags.
+pages, every block scale, the zero tails and the ready tags. That holds while
+the library and the oracle build their rotary (cos, sin) tables with the same
+host C library: both evaluate pow, cos and sin in float64 through the system
+libm (libwf's pool set-up in C++, the oracle through Python's math module) and
+round once to float32. A libm whose results differ in the last bit could move
+a float32 table entry and, through it, an occasional E4M3 code; the attention
+checks below would still pass, the bit-for-bit code check would not.
 
 Attention tolerances (derived, E4M3 P operand): the kernel rounds each
 probability, scaled by a power of two, to E4M3. In the normal range that is a
