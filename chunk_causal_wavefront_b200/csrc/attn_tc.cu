@@ -10,9 +10,12 @@
 //
 // One CTA computes O = softmax(Q K^T / sqrt(d)) V for two 128-row query tiles
 // (q = 0, 1) of one (slot, head), sharing every K/V page it loads:
-//   warp 8 (one lane)  TMA producer: Q0, Q1 once, then for every key tile (one
-//                      128-token page, found through the page table) K and V
-//                      into a two-stage shared-memory ring (128-byte swizzle).
+//   warp 8 (one lane)  TMA producer of Q0, Q1 (once) and, for every key tile
+//                      (one 128-token page, found through the page table), K
+//                      into a shared-memory ring (128-byte swizzle; two stages
+//                      for bf16, three for E4M3).
+//   warp 10 (one lane) TMA producer of V into a ring of the same depth, apart
+//                      from K so that no K load queues behind a V load.
 //   warp 9 (one lane)  tcgen05 issuer, in the order
 //                        S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ...
 //                      S_q = Q_q K^T goes to TMEM columns [128q, 128q+128);
@@ -27,7 +30,9 @@
 //                      the running max grows by more than a threshold (lazy
 //                      rescaling: the exponentials stay below 2^threshold
 //                      otherwise), the only time softmax waits for the previous
-//                      P*V. Only the row max and the exponentials sit between
+//                      P*V. A share of the exponentials runs as a polynomial on
+//                      the FMA pipe (the MUFU unit does 16 per clock per SM).
+//                      Only the row max and the exponentials sit between
 //                      S ready and P ready: the row sum and the correction
 //                      factor are updated after P is handed over, and the
 //                      last-page test is taken before the wait for S. The
@@ -46,11 +51,12 @@
 //         units of 2^(ev_max - 4) and the row sum adds P'_j * 2^(ev_max + 4 - ev_j).
 //         The lazy threshold is 2^4, so P' <= 2^8 stays inside E4M3's range
 //         (448) while small probabilities keep 4 more binades above its
-//         subnormal range. With the MMAs at twice the bf16 rate the two tiles'
-//         exponential phases would overlap on the MUFU unit, so the softmax
-//         warps of a sub-partition take turns on them (one mbarrier per
-//         sub-partition and tile; the turn passes after three quarters of the
-//         row).
+//         subnormal range. P_q lives in shared memory (the tile's 32 KB output
+//         staging block, idle until the epilogue), read by an SS P*V MMA, so
+//         the issuer computes S_q(j+1) as soon as the softmax has read S_q(j)
+//         into registers (an "S read" barrier) instead of after P_q(j)*V: the
+//         MMA latency leaves the softmax's chain. (Turn-taking between the two
+//         tiles' softmax warps on the MUFU unit is kept as an option, off.)
 // Every wait is bounded: on timeout the CTA records WF_ERR_TIMEOUT, the other
 // roles see the abort flag, in-flight copies and MMAs are drained (with a
 // separate, longer bound), pending TMEM stores are waited for, and TMEM is
@@ -73,14 +79,15 @@ constexpr int kBN = 128;              // keys per tile (one page)
 constexpr int kHD = 128;              // head dim
 constexpr int kPageCache = 1024;      // page ids (and FP8 scale exponents) cached in smem
 // Warpgroups 0 and 1 run the softmax of tiles 0 and 1; warpgroup 2 holds the
-// TMA producer (warp 8) and the MMA issuer (warp 9); warps 10-11 only hand
-// their registers over. Launched at 168 registers per thread (384 x 168 =
+// TMA producers (warp 8: Q and K, warp 10: V) and the MMA issuer (warp 9);
+// warp 11 only hands its registers over. Launched at 168 registers per thread (384 x 168 =
 // 64512), warpgroup 2 gives registers to the softmax warpgroups: 96 / 200 for
 // bf16, 80 / 208 for E4M3 (whose softmax also carries the block scales; timed
 // 1.8 % faster than 96 / 200, which is the faster split for bf16).
 constexpr int kThreads = 384;
-constexpr int kProducerWarp = 8;
+constexpr int kProducerWarp = 8;    // Q and K loads
 constexpr int kMmaWarp = 9;
+constexpr int kVProducerWarp = 10;  // V loads
 template <bool kF8> constexpr uint32_t kRegsSoftmax = kF8 ? 208 : 200;
 template <bool kF8> constexpr uint32_t kRegsControl = kF8 ? 80 : 96;
 static_assert(256 * kRegsSoftmax<false> + 128 * kRegsControl<false> <= 384 * 168, "register split");
@@ -96,16 +103,19 @@ struct Fmt {
   // 64-column 128-byte-swizzled halves, E4M3 as one 128-byte-swizzled block.
   static constexpr uint32_t kTile = kF8 ? 16384 : 32768;
   static constexpr uint32_t kHalf = 16384;          // bf16 half / fp8 whole tile
+  // Stages of the K ring and of the V ring: three for E4M3 (16 KB tiles leave
+  // room), two for bf16 (whose rings already fill 128 KB of shared memory).
+  static constexpr int kStages = kF8 ? 3 : 2;
   static constexpr uint32_t kOffQ = 0;                          // Q0, Q1
-  static constexpr uint32_t kOffK = kOffQ + 2 * kTile;          // 2 stages
-  static constexpr uint32_t kOffV = kOffK + 2 * kTile;          // 2 stages
+  static constexpr uint32_t kOffK = kOffQ + 2 * kTile;          // K ring
+  static constexpr uint32_t kOffV = kOffK + kStages * kTile;    // V ring
   // bf16 output staging: the tile's own Q buffer (bf16) or a separate 32 KB
   // buffer per tile (E4M3, whose Q tile is only 16 KB).
-  static constexpr uint32_t kOffStage = kOffV + 2 * kTile;
+  static constexpr uint32_t kOffStage = kOffV + kStages * kTile;
   static constexpr uint32_t kOffBar = kF8 ? kOffStage + 2 * 32768 : kOffStage;
   static constexpr float kLazy = kF8 ? 4.0f : 8.0f;             // rescale threshold (log2)
   static constexpr int kPShift = 4;                             // E4M3 headroom of P'
-  static constexpr int kNumBars = 26;
+  static constexpr int kNumBars = 30;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // TMEM base, abort, 12 ints
   static constexpr uint32_t kOffPages = kOffMisc + 64;
   static constexpr uint32_t kOffExps = kOffPages + kPageCache * 4;   // int16 ek, ev (FP8)
@@ -114,10 +124,10 @@ struct Fmt {
 
 constexpr int kNumBars = Fmt<false>::kNumBars;
 enum Bar {
-  kQFull = 0, kKFull0 = 1, kKEmpty0 = 3, kVFull0 = 5, kVEmpty0 = 7,
-  kSFull0 = 9, kPReady0 = 11, kPVDone0 = 13, kDrain = 15,
-  kTurn0 = 16, kTurn1 = 20,  // E4M3: exponential-phase turns, one per sub-partition and tile
-  kSRead0 = 24               // E4M3: the softmax has read S_q into registers (one per tile)
+  kQFull = 0, kKFull0 = 1, kKEmpty0 = 4, kVFull0 = 7, kVEmpty0 = 10,   // up to 3 stages each
+  kSFull0 = 13, kPReady0 = 15, kPVDone0 = 17, kDrain = 19,
+  kTurn0 = 20, kTurn1 = 24,  // E4M3: exponential-phase turns, one per sub-partition and tile
+  kSRead0 = 28               // E4M3: the softmax has read S_q into registers (one per tile)
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -386,36 +396,58 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(sQ + kTile + F::kHalf, &tq, bars + kQFull, 64, h, row0 + kBM, slot);
         }
       }
-      int nk0 = 0, nk1 = 0, nv0 = 0, nv1 = 0;   // loads issued per stage
+      // K of key tile j goes to stage j % kStages as that stage's fill
+      // j / kStages, behind the S MMAs of tile j - kStages (K empty).
+      int jk_last = -1;                          // last K tile loaded
       for (int j = 0; j < n_tiles; ++j) {
-        const int stg = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
+        const int stg = j % F::kStages;
+        const uint32_t ph = (j / F::kStages) & 1;
         const int phys = j < kPageCache ? page_cache[j] : __ldcg(p.table + kTabPages + j);
         const int rowk = static_cast<int>(p.layer_row0) + ((phys * 2) * p.Hh + h) * p.P;
-        const int rowv = rowk + p.Hh * p.P;
         uint8_t *sK = smem + F::kOffK + stg * kTile;
-        uint8_t *sV = smem + F::kOffV + stg * kTile;
         if (!wait_bar(ctx, kKEmpty0 + stg, ph ^ 1)) break;
         if (j != p.skip_key_tile) {   // test hook: a skipped load leaves its wait to run out
           mbar_arrive_expect_tx(bars + kKFull0 + stg, kTile);
           tma_load_2d(sK, &tkv, bars + kKFull0 + stg, 0, rowk);
           if (!kF8) tma_load_2d(sK + F::kHalf, &tkv, bars + kKFull0 + stg, 64, rowk);
-          if (stg) ++nk1; else ++nk0;
+          jk_last = j;
         }
+      }
+      // Drain: every load this thread issued has landed before the CTA exits.
+      // Loads into one stage complete its phases in order, so waiting for the
+      // phase of the last one issued into each stage covers them all.
+#pragma unroll
+      for (int st = 0; st < F::kStages; ++st) {
+        int jl = jk_last - ((jk_last - st) % F::kStages + F::kStages) % F::kStages;
+        if (jl == p.skip_key_tile) jl -= F::kStages;   // the hook's tile was never loaded
+        if (jl >= 0) drain_wait(ctx, kKFull0 + st, (jl / F::kStages) & 1);
+      }
+      drain_wait(ctx, kQFull, 0);
+    }
+  } else if (warp == kVProducerWarp) {
+    // ---------------------------------------------------------- V producer --
+    // V of key tile j goes to stage j % kStages behind the P*V MMAs of tile
+    // j - kStages (V empty); a separate thread, so that K loads never queue
+    // behind a V load waiting for its stage.
+    if (lane == 0) {
+      int jv_last = -1;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int stg = j % F::kStages;
+        const uint32_t ph = (j / F::kStages) & 1;
+        const int phys = j < kPageCache ? page_cache[j] : __ldcg(p.table + kTabPages + j);
+        const int rowv = static_cast<int>(p.layer_row0) + ((phys * 2 + 1) * p.Hh + h) * p.P;
+        uint8_t *sV = smem + F::kOffV + stg * kTile;
         if (!wait_bar(ctx, kVEmpty0 + stg, ph ^ 1)) break;
         mbar_arrive_expect_tx(bars + kVFull0 + stg, kTile);
         tma_load_2d(sV, &tkv, bars + kVFull0 + stg, 0, rowv);
         if (!kF8) tma_load_2d(sV + F::kHalf, &tkv, bars + kVFull0 + stg, 64, rowv);
-        if (stg) ++nv1; else ++nv0;
+        jv_last = j;
       }
-      // Drain: every load this thread issued has landed before the CTA exits.
-      // Loads into one stage complete its phases in order, so waiting for the
-      // phase of the last one issued covers them all.
-      if (nk0) drain_wait(ctx, kKFull0, (nk0 - 1) & 1);
-      if (nk1) drain_wait(ctx, kKFull0 + 1, (nk1 - 1) & 1);
-      if (nv0) drain_wait(ctx, kVFull0, (nv0 - 1) & 1);
-      if (nv1) drain_wait(ctx, kVFull0 + 1, (nv1 - 1) & 1);
-      drain_wait(ctx, kQFull, 0);
+#pragma unroll
+      for (int st = 0; st < F::kStages; ++st) {
+        const int jl = jv_last - ((jv_last - st) % F::kStages + F::kStages) % F::kStages;
+        if (jl >= 0) drain_wait(ctx, kVFull0 + st, (jl / F::kStages) & 1);
+      }
     }
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- MMA issuer --
@@ -445,9 +477,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t p_lo = desc_lo_sw128(smem_u32(smem + F::kOffStage), 16);
       constexpr uint32_t kPStep = 32768 >> 4;                 // tile 1's P (staging) buffer
       for (int j = 0; kF8 && ok && j < n_tiles; ++j) {
-        const int stg = j & 1, nstg = (j + 1) & 1;
+        const int stg = j % F::kStages, nstg = (j + 1) % F::kStages;
         if (j + 1 < n_tiles) {
-          if (!wait_bar(ctx, kKFull0 + nstg, ((j + 1) >> 1) & 1)) break;
+          if (!wait_bar(ctx, kKFull0 + nstg, ((j + 1) / F::kStages) & 1)) break;
           if (!wait_bar(ctx, kSRead0, j & 1)) break;
           tc_fence_after();
           issue_s<kF8>(tmem + kTmemS, q_lo, k_lo + nstg * kTileStep, hi);
@@ -460,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(bars + kKEmpty0 + nstg);
         }
-        if (!wait_bar(ctx, kVFull0 + stg, (j >> 1) & 1)) break;
+        if (!wait_bar(ctx, kVFull0 + stg, (j / F::kStages) & 1)) break;
         if (!wait_bar(ctx, kPReady0, j & 1)) break;
         tc_fence_after();
         issue_pv_f8_smem(tmem + kTmemO, p_lo, v_lo + stg * kTileStep, hi, j > 0);
@@ -474,15 +506,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bars + kVEmpty0 + stg);
       }
       for (int j = 0; !kF8 && ok && j < n_tiles; ++j) {
-        const int stg = j & 1, nstg = (j + 1) & 1;
+        const int stg = j % F::kStages, nstg = (j + 1) % F::kStages;
         const bool more = j + 1 < n_tiles;
-        if (!wait_bar(ctx, kVFull0 + stg, (j >> 1) & 1)) break;
+        if (!wait_bar(ctx, kVFull0 + stg, (j / F::kStages) & 1)) break;
         if (!wait_bar(ctx, kPReady0, j & 1)) break;
         tc_fence_after();
         issue_pv<kF8>(tmem + kTmemO, tmem + kTmemS, v_lo + stg * kTileStep, hi, j > 0);
         mma_commit(bars + kPVDone0);
         if (more) {
-          if (!wait_bar(ctx, kKFull0 + nstg, ((j + 1) >> 1) & 1)) break;
+          if (!wait_bar(ctx, kKFull0 + nstg, ((j + 1) / F::kStages) & 1)) break;
           tc_fence_after();
           issue_s<kF8>(tmem + kTmemS, q_lo, k_lo + nstg * kTileStep, hi);
           mma_commit(bars + kSFull0);
@@ -523,6 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     float m = -INFINITY, l = 0.0f;
     bool ok = true;
+    int jp = 0;                      // page of tile j inside its chunk (no division in the loop)
     for (int j = 0; j < n_tiles; ++j) {
       float c_j = p.scale_log2;      // log2(e)/sqrt(d) times the FP8 block scales
       float dv = 0.0f;               // FP8: log2 of P's V-scale factor, ev_j - ev_max + 4
@@ -543,7 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Keys past the chunk's length on its last page are masked. Worked out
       // before the wait: after it, the integer division would queue on the
       // MUFU unit behind the other tile's exponentials.
-      const int valid = (j % p.npc == p.npc - 1) ? last_valid : kBN;
+      const int valid = jp == p.npc - 1 ? last_valid : kBN;
+      if (++jp == p.npc) jp = 0;
       ok = __all_sync(0xffffffffu, wait_bar(ctx, kSFull0 + q, j & 1));
       if (!ok) break;
       tc_fence_after();
@@ -660,14 +694,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, wait_bar(ctx, kPVDone0 + q, (j - 1) & 1));
         if (!ok) break;
         tc_fence_after();
+        const float alpha = rescale ? ex2(m - m_use) : 1.0f;
+        const uint64_t a2 = f2(alpha, alpha);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           tmem_ld32(tO + c * 32, o);
           tmem_ld_wait();
           reg_fence32(o);
-          const float alpha = rescale ? ex2(m - m_use) : 1.0f;
-          const uint64_t a2 = f2(alpha, alpha);
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             const uint64_t v = fmul2(f2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
@@ -690,7 +724,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       unf2(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), sum0, sum1);
       float tile_sum = sum0 + sum1;
       if (kF8) tile_sum *= exp2i(-static_cast<int>(dv));   // back to units of P
-      l = l * (rescale ? ex2(m - m_use) : 1.0f) + tile_sum;
+      if (rescale) l *= ex2(m - m_use);   // the MUFU only when the max moved
+      l += tile_sum;
       m = m_use;
     }
     if (ok && n_tiles > 0) {
