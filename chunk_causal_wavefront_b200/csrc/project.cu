@@ -292,8 +292,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
             const float a = __uint_as_float(cur[2 * q]), bb = __uint_as_float(cur[2 * q + 1]);
-            cur[2 * q] = __float_as_uint(a * cs[q].x - bb * cs[q].y);
-            cur[2 * q + 1] = __float_as_uint(a * cs[q].y + bb * cs[q].x);
+            // Each product and sum rounded once, as in the publish kernels.
+            cur[2 * q] = __float_as_uint(__fsub_rn(__fmul_rn(a, cs[q].x), __fmul_rn(bb, cs[q].y)));
+            cur[2 * q + 1] = __float_as_uint(__fadd_rn(__fmul_rn(a, cs[q].y), __fmul_rn(bb, cs[q].x)));
           }
         }
         if (live_page && c == 2) {

@@ -13,8 +13,8 @@
 // One launch covers every live slot of the round (grid row = slot). A thread
 // handles 16-byte vectors (4 fp32 values = 2 rotary pairs) of (slot, token,
 // head) rows, two per iteration: it loads q, k and v with streaming 16-byte
-// loads, rotates q and k with (cos, sin) tables computed on the host in fp64,
-// and issues 16-byte stores to q_rot and to the K and V pages. Consecutive
+// loads, rotates q and k in fp32 (each product and sum rounded once) with
+// (cos, sin) tables computed on the host in fp64 and rounded to fp32, and issues 16-byte stores to q_rot and to the K and V pages. Consecutive
 // threads cover consecutive 16-byte vectors of the [C][heads][d] input rows,
 // so loads are fully coalesced. HBM-bound: 3 reads + 3 writes of every
 // element.
@@ -87,8 +87,8 @@ __device__ __forceinline__ void rope_vec(float *x, int dim0, int tpos, int ypos,
     else if (pr < h0 + h1) cs = __ldg(p.rope_h + ypos * h1 + (pr - h0));
     else cs = __ldg(p.rope_w + xpos * h2 + (pr - h0 - h1));
     const float a = x[2 * i], b = x[2 * i + 1];
-    x[2 * i] = a * cs.x - b * cs.y;
-    x[2 * i + 1] = a * cs.y + b * cs.x;
+    x[2 * i] = __fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y));     // no FMA contraction
+    x[2 * i + 1] = __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x));
   }
 }
 

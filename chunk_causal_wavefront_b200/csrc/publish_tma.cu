@@ -108,7 +108,10 @@ __device__ __forceinline__ void rotate_vec(uint4 &u, const float2 (&cs)[4]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float a = __uint_as_float(w[i] << 16), b = __uint_as_float(w[i] & 0xFFFF0000u);
-    __nv_bfloat162 r = __floats2bfloat162_rn(a * cs[i].x - b * cs[i].y, a * cs[i].y + b * cs[i].x);
+    // Each product and sum rounded once (no contraction into FMAs), then one
+    // rounding to bf16: the published values are a function of the inputs alone.
+    __nv_bfloat162 r = __floats2bfloat162_rn(__fsub_rn(__fmul_rn(a, cs[i].x), __fmul_rn(b, cs[i].y)),
+                                             __fadd_rn(__fmul_rn(a, cs[i].y), __fmul_rn(b, cs[i].x)));
     w[i] = *reinterpret_cast<uint32_t *>(&r);
   }
   u = make_uint4(w[0], w[1], w[2], w[3]);

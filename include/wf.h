@@ -148,7 +148,9 @@ wf_status wf_kv_pool_create(const wf_pool_config *cfg, void *dev_mem, size_t byt
 
 /* Publish one layer's K/V for every live slot of the current round (early
  * publication after QKV + RoPE, Method section): applies the 3D rotary
- * embedding to q and k (fp32 math, one rounding), writes q_rot, scatters
+ * embedding to q and k (fp32 math with each product and sum rounded once,
+ * (cos, sin) from the host's float64 cos and sin rounded to fp32; then one
+ * rounding to the pool's dtype), writes q_rot, scatters
  * rotated K and V into the slots' pages (rows past C in a chunk's last page
  * are zeroed) and stamps each written page's ready tag.
  *   q, k, v : inputs, [S+1][C][heads][d]; rows of slots that are not live in

@@ -12,8 +12,8 @@ This test models those float32 steps with NumPy (IEEE round-to-nearest-even
 adds, fused multiply-adds evaluated exactly in float64 and rounded once) and
 checks them against numpy.exp2 over the whole input range the softmax can
 produce (at most 8 above the running maximum, down to -inf):
-  * degree 2: relative error within 1.8e-3, far below E4M3's half unit 2^-4;
-  * degree 3: relative error within 8e-5, far below bf16's half unit 2^-9;
+  * degree 2: relative error within 1.8e-3, far below E4M3's unit roundoff 2^-4;
+  * degree 3: relative error within 8e-5, far below bf16's unit roundoff 2^-8;
   * -inf (masked keys) and anything below -126 give a finite non-negative
     value below 2^-125, which is zero after rounding to E4M3 at every block
     scale the kernel applies, and nothing next to a row sum of at least 1.

@@ -85,11 +85,13 @@ def _sample_rows(C, n, seed):
     return np.array(sorted(rows))
 
 
-@pytest.mark.parametrize("name,heads", [("wan13b_bf16", (0, 11)), ("wan14b_bf16", (17,))])
+@pytest.mark.parametrize("name,heads", [("wan13b_bf16", (0, 11)), ("wan14b_bf16", (17,)),
+                                        ("wan13b_5step_bf16", (3,)), ("wan13b_bf16_rf", (5,))])
 def test_full_size_all_rows(name, heads):
     # Every query row of every live slot of the listed heads: 19 tile pairs
     # per (slot, head) in the full grid's launch order, against the oracle.
-    cfg = wf_inputs.CONFIGS[name]
+    cfg = (wf_inputs.CONFIGS["wan13b_bf16"].replace(mask="rf") if name.endswith("_rf")
+           else wf_inputs.CONFIGS[name])
     ro = _steady(cfg)
     _compare(ro, heads, rows=None, name=name + "_all_rows")
     ro.close()

@@ -235,6 +235,24 @@ def test_fp8_full_size_sampled(name):
     assert rec
 
 
+def test_fp8_full_size_all_rows():
+    # Every query row of every live slot of one head at full size (19 tile
+    # pairs per slot in the launch configuration bench.py times).
+    cfg = wf_inputs.CONFIGS["wan13b_bf16"]
+    ro = Fp8Rollout(cfg, page_seed=8)
+    rec = []
+    for k in range(cfg.steady_round() + 1):
+        ro.publish()
+        if k == cfg.steady_round():
+            ro.attention()
+            assert ro.pool.check_status() == 0
+            ro.check_publish(heads=[4])
+            ro.check_attention(heads=[4], rows=None, record=rec)
+        ro.pool.advance()
+    ro.close()
+    assert len(rec) == cfg.num_slots
+
+
 def test_fp8_long_context_past_page_cache():
     # 29 chunks x 37 pages = 1073 key tiles: page ids and K/V scale exponents
     # past the 1024 cached in shared memory are read through the page table.

@@ -1,14 +1,16 @@
 """GPU parity of wf_publish_kv: rotary embedding and paged scatter.
 
 Page placement and V contents are checked bit-exactly against the oracle's
-page-table model; rotated K and q_rot against the float64 oracle rotation
-within one bf16 ulp (fp32: 1e-5 absolute), at the full 1.3B-shaped size."""
+page-table model; rotated K and q_rot bit for bit against the oracle's float32
+rotation rounded once to the pool's dtype, and within one bf16 ulp (fp32: 1e-5
+absolute) of the float64 rotation, at the full 1.3B-shaped size."""
 import numpy as np
 import pytest
 import torch
 
 import wf_inputs
 from oracle import wf_oracle as O
+from oracle import wf_fp8 as F8
 from wf_test_utils import Rollout, bf16_ulp, min_pages, tensor_f64, to_f64
 
 pytestmark = pytest.mark.gpu
@@ -63,6 +65,15 @@ def _check_round(ro: Rollout, layer: int = 0, full_rope_check: bool = True):
             else:
                 assert np.abs(gk - k64).max() <= 1e-5, p
                 assert np.abs(gq - q64).max() <= 1e-5, p
+            if c.rope:
+                # bit for bit: the oracle's float32 rotation (each product and
+                # sum rounded once), then one rounding to the pool's dtype
+                for got, x in ((gk, k), (gq, q)):
+                    r32 = F8.rope_3d_f32(to_f64(x, c.dtype).astype(np.float32), chunk,
+                                         c.frames_per_chunk, c.grid_h, c.grid_w, c.rope_split,
+                                         c.rope_base).astype(np.float64)
+                    want = O.round_bf16(r32) if c.dtype == "bf16" else r32
+                    assert np.array_equal(got, want), (p, int((got != want).sum()))
             if not c.rope:
                 assert np.array_equal(gk, k64) and np.array_equal(gq, q64)
 

@@ -18,6 +18,7 @@ import torch
 import wf_inputs
 from wf_inputs import WorkloadConfig, bf16_bits_to_f64
 from oracle import wf_oracle as O
+from oracle import wf_fp8 as F8
 
 
 def pool_config(cfg: WorkloadConfig, **over):
@@ -148,17 +149,32 @@ class Rollout:
                                        mask=self.cfg.mask)
 
     def oracle_out_bf16_operands(self, heads: Sequence[int], rows=None, layer: int = 0):
-        """Oracle attention on operands rounded to the published bf16 format.
+        """Oracle attention on the operands the pool publishes: q and k rotated
+        in float32 with each product and sum rounded once (rope_3d_f32, the
+        oracle's rule for published rotations), then rounded to bf16 by the
+        oracle itself (round_bf16), the storage format of q_rot and the K pages.
+        Nothing here is read back from the GPU."""
+        c, hs = self.cfg, list(heads)
+        if c.dtype != "bf16":
+            raise ValueError("bf16 pools only")
 
-        The oracle rotates q and k in float64 and rounds them to bf16 itself
-        (round_bf16), modelling the storage format of q_rot and the K pages;
-        nothing here is read back from the GPU.
-        """
-        q_rot, keys, vals = self.oracle_tensors(heads, layer)
-        q_rot = {s: O.round_bf16(x) for s, x in q_rot.items()}
-        keys = {c: O.round_bf16(x) for c, x in keys.items()}
+        def pub(bits, chunk):
+            x = to_f64(bits, c.dtype)[:, hs]
+            if c.rope:
+                x = F8.rope_3d_f32(x.astype(np.float32), chunk, c.frames_per_chunk, c.grid_h,
+                                   c.grid_w, c.rope_split, c.rope_base).astype(np.float64)
+            return O.round_bf16(x)
+
+        q_rot, keys, vals = {}, {}, {}
+        for s, (q, k, v, chunk) in self.live[layer].items():
+            q_rot[s] = pub(q, chunk)
+        for p in self.layout():
+            kb, vb = (self.stored[layer][p.chunk] if p.slot is None
+                      else self.live[layer][p.slot][1:3])
+            keys[p.chunk] = pub(kb, p.chunk)
+            vals[p.chunk] = to_f64(vb, c.dtype)[:, hs]
         return O.attention_slot_prefix(q_rot, keys, vals, self.layout(), rows=rows,
-                                       mask=self.cfg.mask)
+                                       mask=c.mask)
 
     def close(self):
         self.pool.close()
@@ -168,14 +184,21 @@ class Rollout:
 
 BF16_ABS, BF16_REL = 2e-2, 1e-2
 F32_ABS = 1e-5
-# With 5% of K rows scaled x8 the softmax is sharply peaked and rounding the
-# rotated q and k to bf16 (the published format) moves each dominant logit by
-# about 8 * 2^-9; near-tied dominant keys then shift outputs of size ~3 by a few
-# 1e-2 against the exact float64 result, whatever the kernel does. So every
-# bf16 case is checked twice: against the oracle run on bf16-rounded q_rot and
-# K (the kernel's own error: max-abs 2e-2, rel-L2 1e-2), and against the exact
-# oracle (rel-L2 1e-2; max-abs 2e-2 on top of the rounding effect
-# |O_exact - O_bf16| that the oracle itself computes).
+# Every bf16 case is checked twice.
+#  * Against the oracle run on the published operands (q and k rotated in
+#    float32 and rounded to bf16 by the oracle, the values the publish tests
+#    find bit for bit in q_rot and the K pages): this is the kernel's own
+#    error. Per element, |O - O_pub| <= 2e-2 + u |O_pub|, and rel-L2 <= 1e-2.
+#    u = 2^-8 is bf16's unit roundoff (8-bit significand): the output is
+#    stored in bf16 (the pages run BF16), and at |O| in [4, 8), where the x8
+#    outlier keys put some outputs, rounding alone moves it by up to 2^-6.
+#  * Against the exact float64 oracle: rel-L2 <= 1e-2, and per element
+#    max-abs 2e-2 on top of the rounding effect |O_exact - O_pub| that the
+#    oracle itself computes. With 5% of K rows scaled x8 the softmax is sharply
+#    peaked and rounding q and k to bf16 moves each dominant logit by about
+#    8 * 2^-9; near-tied dominant keys then shift outputs of size ~3 by a few
+#    1e-2 against the exact result, whatever the kernel does.
+BF16_U = 2.0 ** -8
 
 
 def log_parity(name, **kw):
@@ -190,7 +213,8 @@ def compare_with_oracle(ro: "Rollout", heads, rows=None, gpu_operands=True, name
     float64 oracle for the given heads and rows, at the tolerances above."""
     c = ro.cfg
     want = ro.oracle_out(heads, rows, layer)
-    want_g = ro.oracle_out_bf16_operands(heads, rows, layer) if gpu_operands else None
+    want_g = (ro.oracle_out_bf16_operands(heads, rows, layer)
+              if gpu_operands and c.dtype == "bf16" else None)
     out = tensor_f64(ro.out)
     live = {p.slot for p in ro.layout() if p.slot is not None}
     for s in range(c.num_slots):
@@ -209,14 +233,16 @@ def compare_with_oracle(ro: "Rollout", heads, rows=None, gpu_operands=True, name
         if want_g is not None:
             rec.update(max_abs_bf16_operands=float(np.abs(got_s - want_g[s]).max()),
                        rel_l2_bf16_operands=rel_l2(got_s, want_g[s]),
-                       rounding_effect=float(np.abs(want_g[s] - want[s]).max()))
+                       rounding_effect=float(np.abs(want_g[s] - want[s]).max()),
+                       max_abs_out=float(np.abs(want_g[s]).max()))
         log_parity(name, **rec)
         assert r <= BF16_REL, (s, rec)
         if want_g is None:
             assert err <= BF16_ABS, (s, rec)
         else:
             assert (np.abs(got_s - want[s]) <= BF16_ABS + np.abs(want_g[s] - want[s])).all(), (s, rec)
-            assert rec["max_abs_bf16_operands"] <= BF16_ABS, (s, rec)
+            dev = np.abs(got_s - want_g[s])
+            assert (dev <= BF16_ABS + BF16_U * np.abs(want_g[s])).all(), (s, rec)
             assert rec["rel_l2_bf16_operands"] <= BF16_REL, (s, rec)
             if c.k_outlier_frac == 0:
                 assert err <= BF16_ABS, (s, rec)
