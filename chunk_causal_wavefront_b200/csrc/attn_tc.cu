@@ -55,7 +55,12 @@
 //         staging block, idle until the epilogue), read by an SS P*V MMA, so
 //         the issuer computes S_q(j+1) as soon as the softmax has read S_q(j)
 //         into registers (an "S read" barrier) instead of after P_q(j)*V: the
-//         MMA latency leaves the softmax's chain. (Turn-taking between the two
+//         MMA latency leaves the softmax's chain. The softmax still waits
+//         for P_q(j-1)*V before it overwrites P_q; that wait keeps the two
+//         tiles' softmax warps of a sub-partition out of phase, so their
+//         exponentials do not contend for MUFU and issue slots (computing the
+//         whole row before the wait, or issuing the MMAs in the order their
+//         inputs become ready, measured slower). (Turn-taking between the two
 //         tiles' softmax warps on the MUFU unit is kept as an option, off.)
 // Every wait is bounded: on timeout the CTA records WF_ERR_TIMEOUT, the other
 // roles see the abort flag, in-flight copies and MMAs are drained (with a
