@@ -21,9 +21,13 @@ from wf_test_utils import compare_with_oracle as _compare
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("mask", ["wf", "rf"])
-def test_tiny_f32_every_round(mask):
-    cfg = wf_inputs.CONFIGS["tiny_f32"].replace(mask=mask)
+@pytest.mark.parametrize("cfg", [
+    wf_inputs.CONFIGS["tiny_f32"],
+    wf_inputs.CONFIGS["tiny_f32"].replace(mask="rf"),
+    # the largest stage count the ABI accepts: 17 live query slots
+    wf_inputs.CONFIGS["tiny_f32"].replace(num_stages=16, rounds=24),
+], ids=["wf", "rf", "S16"])
+def test_tiny_f32_every_round(cfg):
     ro = Rollout(cfg, page_seed=0)
     for k in range(cfg.rounds + 3):
         ro.publish(0)
@@ -49,7 +53,13 @@ SMALL_BF16 = wf_inputs.CONFIGS["wan13b_bf16"].replace(
     SMALL_BF16.replace(mask="rf"),
     SMALL_BF16.replace(mask="rf", anchor_chunks=0, history_chunks=1, chunk_tokens=3 * 4 * 11,
                        frames_per_chunk=3, grid_h=4, grid_w=11),
-], ids=["S3_C300", "noanchor_C132", "S1_C128", "C1", "rf_S3_C300", "rf_noanchor_C132"])
+    # the largest stage count the ABI accepts: 17 live query slots
+    SMALL_BF16.replace(num_stages=16, chunk_tokens=130, grid_h=10, grid_w=13, history_chunks=3,
+                       rounds=24),
+    SMALL_BF16.replace(num_stages=16, chunk_tokens=130, grid_h=10, grid_w=13, history_chunks=3,
+                       rounds=24, mask="rf"),
+], ids=["S3_C300", "noanchor_C132", "S1_C128", "C1", "rf_S3_C300", "rf_noanchor_C132",
+        "S16_C130", "rf_S16_C130"])
 def test_bf16_every_round_small(cfg):
     ro = Rollout(cfg, page_seed=4)
     for k in range(cfg.steady_round() + 3):

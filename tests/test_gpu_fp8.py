@@ -187,9 +187,16 @@ SMALL = wf_inputs.CONFIGS["wan13b_bf16"].replace(
     grid_h=10, grid_w=30, rounds=10)
 
 
-@pytest.mark.parametrize("mask", ["wf", "rf"])
-def test_fp8_small_every_round(mask):
-    cfg = SMALL.replace(mask=mask)
+# The largest stage count the ABI accepts (WF_MAX_STAGES = 16: 17 live query
+# slots, every per-slot array of the launch parameters full), with a ragged
+# two-tile chunk (130 = 128 + 2 rows).
+MAX_STAGES = SMALL.replace(num_stages=16, chunk_tokens=130, grid_h=10, grid_w=13, history_chunks=3,
+                          rounds=24)
+
+
+@pytest.mark.parametrize("cfg", [SMALL, SMALL.replace(mask="rf"), MAX_STAGES],
+                         ids=["wf", "rf", "max_stages"])
+def test_fp8_small_every_round(cfg):
     ro = Fp8Rollout(cfg, page_seed=3)
     for k in range(cfg.steady_round() + 3):
         ro.publish()

@@ -29,7 +29,7 @@ def pool_config(cfg: WorkloadConfig, **over):
               num_layers=cfg.num_layers, dtype=cfg.dtype, rope=cfg.rope,
               frames_per_chunk=cfg.frames_per_chunk, grid_h=cfg.grid_h, grid_w=cfg.grid_w,
               rope_split=cfg.rope_split if cfg.rope else (0, 0, 0), rope_base=cfg.rope_base,
-              max_rounds=max(cfg.rounds + 1, 16), num_pages=0, mask=cfg.mask)
+              max_rounds=max(cfg.rounds, cfg.steady_round()) + 8, num_pages=0, mask=cfg.mask)
     kw.update(over)
     return make_config(**kw)
 
